@@ -1,0 +1,179 @@
+"""fp64 CPU oracle for the MLA prefill core and its output projection.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may use it; the product library never does.
+
+The arithmetic lives in ``mla_oracle.c`` (plain loops, double precision, a
+two-pass exact softmax). This module only compiles that file with gcc,
+loads it with ctypes and marshals numpy / torch arrays. It shares nothing
+with the CUDA path: the same seeded inputs are handed to both, and neither
+imports the other.
+
+What it follows: page "Kimi K2 · Mix and project", code excerpts
+modeling_deepseek.py 799-840 (query/key assembly, scaled scores, additive
+mask, fp32 softmax over keys, value mix) and 848-852 (head merge, o_proj).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmla_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/libmla_oracle.so`` (gcc, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            u16p = ctypes.POINTER(ctypes.c_uint16)
+            f64p = ctypes.POINTER(ctypes.c_double)
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            u8p = ctypes.POINTER(ctypes.c_uint8)
+            lib.mla_oracle_attn_rows.restype = ctypes.c_int
+            lib.mla_oracle_attn_rows.argtypes = [
+                u16p, u16p, u16p, u16p, u16p, u16p, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, i64p,
+                ctypes.c_int64, f64p, f64p, u8p]
+            lib.mla_oracle_oproj_rows.restype = ctypes.c_int
+            lib.mla_oracle_oproj_rows.argtypes = [
+                f64p, u16p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, f64p]
+            lib.mla_oracle_num_threads.restype = ctypes.c_int
+            lib.mla_oracle_set_num_threads.argtypes = [ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_load().mla_oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().mla_oracle_set_num_threads(int(n))
+
+
+def _bf16_bits(x) -> np.ndarray:
+    """bf16 torch tensor -> contiguous uint16 numpy array of its bit patterns."""
+    import torch
+    if isinstance(x, torch.Tensor):
+        if x.dtype != torch.bfloat16:
+            raise TypeError(f"expected a bf16 tensor, got {x.dtype}")
+        return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16)
+                                    .numpy().view(np.uint16))
+    a = np.asarray(x)
+    if a.dtype != np.uint16:
+        raise TypeError("expected bf16 bit patterns as uint16")
+    return np.ascontiguousarray(a)
+
+
+def bf16_to_f64(x) -> np.ndarray:
+    """Exact widening of a bf16 tensor (or its uint16 bits) to float64."""
+    bits = _bf16_bits(x).astype(np.uint32) << 16
+    return bits.view(np.float32).astype(np.float64)
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def attn_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, rows=None,
+              want_probs=False):
+    """Merged head outputs ``attn[b, i, h*Dv + e]`` for the requested rows.
+
+    Tensors are bf16 with shapes q_nope/k_nope [B,H,T,Dn], q_pe [B,H,T,Dr],
+    k_pe [B,1,T,Dr], v [B,H,T,Dv], mask [B,1,T,T] or None (None = causal).
+    ``rows`` is a sequence of (b, i) pairs, or None for every row in order.
+    ``softmax_scale`` is widened from fp32 to double, the precision the
+    kernels receive it in.
+
+    Returns ``(out [R, H*Dv] float64, fully_masked [R, H] bool[, probs])``.
+    """
+    B, H, T, Dn = q_nope.shape
+    Dr = q_pe.shape[-1]
+    Dv = v.shape[-1]
+    if tuple(q_pe.shape) != (B, H, T, Dr) or tuple(k_nope.shape) != (B, H, T, Dn):
+        raise ValueError("q_pe / k_nope shape mismatch")
+    if tuple(k_pe.shape) != (B, 1, T, Dr) or tuple(v.shape) != (B, H, T, Dv):
+        raise ValueError("k_pe / v shape mismatch")
+    if mask is not None and tuple(mask.shape) != (B, 1, T, T):
+        raise ValueError("mask must be [B,1,T,T]")
+    if rows is None:
+        rb = np.repeat(np.arange(B, dtype=np.int64), T)
+        ri = np.tile(np.arange(T, dtype=np.int64), B)
+    else:
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+        rb = np.ascontiguousarray(rows[:, 0])
+        ri = np.ascontiguousarray(rows[:, 1])
+    R = rb.shape[0]
+    arrays = [_bf16_bits(t) for t in (q_nope, q_pe, k_nope, k_pe, v)]
+    m = _bf16_bits(mask) if mask is not None else None
+    out = np.zeros((R, H * Dv), dtype=np.float64)
+    probs = np.zeros((R, H, T), dtype=np.float64) if want_probs else None
+    fm = np.zeros((R, H), dtype=np.uint8)
+    scale = float(np.float32(softmax_scale))
+    rc = _load().mla_oracle_attn_rows(
+        *[_ptr(a, ctypes.c_uint16) for a in arrays],
+        _ptr(m, ctypes.c_uint16) if m is not None else None,
+        ctypes.c_int64(T), B, H, T, Dn, Dr, Dv, scale,
+        _ptr(rb, ctypes.c_int64), _ptr(ri, ctypes.c_int64), ctypes.c_int64(R),
+        _ptr(out, ctypes.c_double),
+        _ptr(probs, ctypes.c_double) if probs is not None else None,
+        _ptr(fm, ctypes.c_uint8))
+    if rc != 0:
+        raise RuntimeError(f"oracle attn_rows failed ({rc})")
+    if want_probs:
+        return out, fm.astype(bool), probs
+    return out, fm.astype(bool)
+
+
+def oproj_rows(attn: np.ndarray, W_o) -> np.ndarray:
+    """``attn [R, K] float64 . W_o^T`` with W_o bf16 ``[N, K]`` -> [R, N] float64."""
+    a = np.ascontiguousarray(np.asarray(attn, dtype=np.float64))
+    w = _bf16_bits(W_o)
+    N, K = w.shape
+    if a.ndim != 2 or a.shape[1] != K:
+        raise ValueError("attn must be [R, K] with K = W_o.shape[1]")
+    R = a.shape[0]
+    out = np.zeros((R, N), dtype=np.float64)
+    rc = _load().mla_oracle_oproj_rows(_ptr(a, ctypes.c_double),
+                                       _ptr(w, ctypes.c_uint16),
+                                       ctypes.c_int64(R), N, K,
+                                       _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle oproj_rows failed ({rc})")
+    return out
+
+
+def attn_oproj_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, W_o,
+                    rows=None):
+    """Full path for the requested rows: attention, head merge, o_proj.
+
+    Returns ``(out [R, N] float64, fully_masked_row [R] bool)``; a row is
+    flagged when any of its heads had no allowed key.
+    """
+    attn, fm = attn_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale,
+                         rows=rows)
+    return oproj_rows(attn, W_o), fm.any(axis=1)
