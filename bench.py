@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the MLA prefill + o_proj path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step is one pass of the whole path over one batch: the attention kernel
+(all 64 heads, merged heads written to HBM) followed by the o_proj GEMM, both
+through the library's C ABI. Inputs are seeded synthetic tensors of the
+workload's shape, resident in HBM before the timed region. L2 is flushed
+(256 MiB write) between timed steps, outside the per-step CUDA events.
+
+FLOPs are counted causally: B*64*P*2*(192+128) + 2*B*T*8192*7168, with P the
+number of (query, key) pairs the mask allows per (batch, head).
+
+With N > 1 (launched by torchrun) every rank runs its own independent batch
+on its own GPU (weak scaling, no collective on the data path); the timed
+region is bracketed by a barrier and a device synchronize, and the time is
+the max over ranks.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of rows of the
+same workload (rank 0 only), as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA prefill+o_proj TFLOP/s (causal FLOPs) and % of B200 BF16 tensor peak"
+DEFAULT_WORKLOAD = "b1_t4096_causal"
+H, DQK, DV, D_MODEL, K_OPROJ = 64, 192, 128, 7168, 8192
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+# ---------------------------------------------------------------- FLOP counts
+def allowed_pairs(B, T, valid_len=None):
+    """(query, key) pairs the mask allows, summed over the batch (per head)."""
+    if valid_len is None:
+        return B * T * (T + 1) // 2
+    total = 0
+    for L in valid_len:
+        L = int(L)
+        total += L * (L + 1) // 2 + (T - L) * L
+    return total
+
+
+def attn_flops(B, T, valid_len=None):
+    return H * allowed_pairs(B, T, valid_len) * 2 * (DQK + DV)
+
+
+def oproj_flops(M):
+    return 2 * M * K_OPROJ * D_MODEL
+
+
+def row_flops(i, T):
+    """Causal FLOPs of one query row (all heads) plus its o_proj row."""
+    return H * (i + 1) * 2 * (DQK + DV) + 2 * K_OPROJ * D_MODEL
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(name):
+    p = os.path.join(ROOT, "mla_causal_attention_attn_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_source_sha(kernel_file)
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and parts[0] == kernel_file and parts[1] == workload \
+                    and parts[2] == sha:
+                return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mla_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_rows_timed(d, rows, T):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attn_oproj_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], d["mask"],
+                           d["softmax_scale"], d["W_o"], rows=rows)
+    dt = time.perf_counter() - t0
+    fl = sum(row_flops(i, T) for _, i in rows)
+    return dt, fl
+
+
+def spread_rows(B, T, n):
+    rows = []
+    for k in range(n):
+        b = k % B
+        i = int(round((k + 0.5) * T / n)) % T
+        rows.append((b, i))
+    return rows
+
+
+def calibrated_rows(d, B, T, target_s):
+    """Row sample whose oracle run takes about target_s seconds."""
+    probe = spread_rows(B, T, 4)
+    dt, _ = oracle_rows_timed(d, probe, T)
+    n = max(4, min(4096, int(4 * target_s / max(dt, 1e-3))))
+    return spread_rows(B, T, n)
+
+
+def cpu_baseline(d, w, target_s=15.0):
+    import oracle
+    rows = calibrated_rows(d, w.B, w.T, target_s)
+    dt, fl = oracle_rows_timed(d, rows, w.T)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(rows)} query rows (all 64 heads + o_proj) of {w.name}, "
+                      f"spread evenly over t; {dt:.1f} s of fp64 C/OpenMP"}
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from mla_causal_attention_attn_b200 import inputs
+    d = inputs.make_workload(w)
+    per_step = min(8.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = calibrated_rows(d, w.B, w.T, per_step)
+    for _ in range(args.warmup):
+        oracle_rows_timed(d, rows, w.T)
+    tot_t, tot_f = 0.0, 0
+    for _ in range(args.steps):
+        dt, fl = oracle_rows_timed(d, rows, w.T)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"{len(rows)} query rows (all 64 heads + o_proj) of {w.name} per step, "
+              f"spread evenly over t")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, flushed=False),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, flushed=True):
+    return {
+        "workload": w.name, "B": w.B, "T": w.T, "heads": H,
+        "qk_head_dim": "128 nope + 64 rope (rope key shared by all heads)", "v_head_dim": DV,
+        "o_proj": "8192 -> 7168", "mask": "causal + key padding [B,1,T,T]" if w.key_padding
+        else "causal (implicit)", "q_scale": w.q_scale,
+        "l2": "flushed between timed steps (256 MiB write, outside the step events)"
+        if flushed else "n/a",
+        "parallelism": "independent batch per GPU (no collective)",
+    }
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from mla_causal_attention_attn_b200 import binding, inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.load()
+    d = inputs.make_workload(w, seed=rank)
+    names = ["q_nope", "q_pe", "k_nope", "k_pe", "v"] + (["mask"] if d["mask"] is not None else [])
+    g = {k: d[k].to(dev) for k in names}
+    W = d["W_o"].to(dev)
+    B, T = w.B, w.T
+    ws_attn = torch.empty(binding.attn_prefill_workspace_bytes(B, T, d["mask"] is not None) or 16,
+                          dtype=torch.uint8, device=dev)
+    attn = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    scale = d["softmax_scale"]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                             mask=g.get("mask"), softmax_scale=scale, out=attn,
+                             workspace=ws_attn, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        binding.o_proj(attn, W, out=out, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, word = binding.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(gpu_uuid(dev)) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    st, word = binding.device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+
+    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    oproj_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [a + b for a, b in zip(attn_ms, oproj_ms)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    vl = d["valid_len"].tolist() if d["valid_len"] is not None else None
+    fa = attn_flops(B, T, vl)
+    fo = oproj_flops(B * T)
+    flops_step = fa + fo
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    # e2e through mla_attn_oproj from pinned host buffers (W_o stays resident)
+    e2e = None
+    if not args.no_e2e:
+        host = {k: d[k].pin_memory() for k in names}
+        out_h = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16).pin_memory()
+        ws_f = torch.empty(binding.attn_oproj_workspace_bytes(B, T, d["mask"] is not None),
+                           dtype=torch.uint8, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * out_h.element_size()
+        n_e2e = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            for k in names:
+                g[k].copy_(host[k], non_blocking=True)
+            binding.attn_oproj(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"], W,
+                               mask=g.get("mask"), softmax_scale=scale, out=out,
+                               workspace=ws_f, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * flops_step * n_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": e2e_ms / n_e2e, "call": "mla_attn_oproj",
+               "note": "per step: pinned H2D of the activations (and mask), the fused call, "
+                       "D2H of the output; W_o resident like any weight"}
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    a_avg = statistics.mean(attn_ms)
+    o_avg = statistics.mean(oproj_ms)
+    kern = {"attn": (fa, a_avg, "attn_prefill.cu", "mla_attn_prefill_kernel"),
+            "oproj": (fo, o_avg, "oproj_gemm.cu", "oproj_gemm_kernel")}
+    dom = max(kern, key=lambda k: kern[k][1])
+    f_dom, t_dom, src_dom, kname = kern[dom]
+    achieved = f_dom / (t_dom * 1e-3) / 1e12
+    roofline = {"kernel": kname, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "peak_source": f"{peak_src} bf16 burst",
+                "traffic": recorded_traffic(src_dom, w.name),
+                "per_launch_flops": f_dom, "avg_launch_ms": t_dom}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(d, w)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: activations N(0,1), W_o N(0,0.02))",
+        "config": workload_config(w),
+        "pct_of_peak": {"measured_bf16_burst": 100 * value / peaks["bf16_tflops"],
+                        "measured_bf16_sustained": 100 * value / peaks["bf16_tflops_sustained"],
+                        "datasheet_dense_bf16": 100 * value / DATASHEET_BF16_TFLOPS,
+                        "peak_source": peak_src},
+        "kernels_ms": {"attn": a_avg, "oproj": o_avg},
+        "flops_per_step": {"attn": fa, "oproj": fo},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": args.steps * (2 + (1 if d["mask"] is not None else 0)),
+        "wall_s_timed_region": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from mla_causal_attention_attn_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA prefill attention + o_proj library
+ * (libmla_b200.so).
+ *
+ * What it computes is the attention core and output projection of one Kimi K2
+ * multi-head latent attention block during prefill, as defined on the page
+ * "Kimi K2 · Mix and project" (code excerpts modeling_deepseek.py 799-840 and
+ * 848-852) with the dimensions of the model configuration printed on
+ * "Kimi K2 · Block input" (num_attention_heads 64, qk_nope_head_dim 128,
+ * qk_rope_head_dim 64, v_head_dim 128, hidden_size 7168):
+ *
+ *   s[b,h,i,j] = softmax_scale * ( q_nope[b,h,i,:] . k_nope[b,h,j,:]
+ *                                + q_pe[b,h,i,:]   . k_pe[b,0,j,:] ) + M[b,0,i,j]
+ *   p[b,h,i,:] = softmax over j of s[b,h,i,:]     (fp32)
+ *   attn[b,i,h*128+e] = sum_j p[b,h,i,j] v[b,h,j,e]     (heads merged)
+ *   out[b,i,n] = sum_k attn[b,i,k] W_o[n,k]             (o_proj, no bias)
+ *
+ * Conventions shared by every call:
+ *  - Element type: bf16, passed as its 16-bit pattern (mla_bf16). All tensors
+ *    are dense, row-major, in the layouts stated per argument.
+ *  - Memory: every pointer is a device pointer on the current CUDA device.
+ *    The caller allocates and frees everything, workspaces included; the
+ *    library never allocates device memory.
+ *  - Alignment: every tensor pointer and the workspace must be 16-byte
+ *    aligned (TMA), the mask 2-byte aligned; otherwise MLA_ERR_MISALIGNED.
+ *  - Streams: work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and the call returns without synchronising. Only
+ *    mla_device_status() synchronises.
+ *  - Errors: every argument is checked before anything is launched; errors
+ *    are returned, never thrown or printed. A kernel that gives up on an
+ *    internal bounded wait records MLA_ERR_TIMEOUT in a device status word that
+ *    mla_device_status() reads.
+ *  - Device: compute capability 10.0 (B200, sm_100a) only; otherwise
+ *    MLA_ERR_UNSUPPORTED_DEVICE.
+ *  - Threads: calls are thread-safe; the library holds no per-call state.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+/* Model dimensions (fixed at compile time; no other values are accepted). */
+#define MLA_NUM_HEADS 64
+#define MLA_QK_NOPE_DIM 128
+#define MLA_QK_ROPE_DIM 64
+#define MLA_V_DIM 128
+#define MLA_OPROJ_IN 8192 /* MLA_NUM_HEADS * MLA_V_DIM */
+#define MLA_HIDDEN 7168
+
+typedef uint16_t mla_bf16; /* bit pattern of a bfloat16 value */
+struct CUstream_st;
+typedef struct CUstream_st* mla_stream_t; /* same type as cudaStream_t */
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,        /* a required pointer is NULL, or a scalar is not finite */
+  MLA_ERR_SHAPE = -2,              /* B, T or M out of range, or mask_ld < T */
+  MLA_ERR_MISALIGNED = -3,         /* a tensor pointer not 16-byte aligned (mask: 2-byte) */
+  MLA_ERR_UNSUPPORTED_DEVICE = -4, /* current device is not compute capability 10.0 */
+  MLA_ERR_WORKSPACE = -5,          /* workspace missing or smaller than required */
+  MLA_ERR_CUDA = -6,               /* a CUDA runtime/driver call or kernel launch failed */
+  MLA_ERR_TIMEOUT = -7             /* a kernel gave up on a bounded internal wait */
+} mla_status_t;
+
+/*
+ * Workspace bytes mla_attn_prefill needs: 0 when has_mask == 0; otherwise
+ * B * ceil(T/128)^2 bytes for the per-tile mask classes. Returns 0 for B < 1
+ * or T < 1.
+ */
+size_t mla_attn_prefill_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * MLA prefill attention for all 64 heads, heads merged
+ * (page "Kimi K2 · Mix and project", excerpt modeling_deepseek.py 799-840:
+ * query/key assembly from the non-rotary and rotary parts, scores scaled by
+ * softmax_scale, additive mask, fp32 softmax over keys, value mix; plus the
+ * transpose/reshape of excerpt 848-852).
+ *
+ *   q_nope       [B, 64, T, 128]  non-rotary query parts
+ *   q_pe         [B, 64, T, 64]   rotary query parts (already rotated)
+ *   k_nope       [B, 64, T, 128]  non-rotary key parts
+ *   k_pe_shared  [B, 1,  T, 64]   rotary key, one tensor shared by all heads
+ *   v            [B, 64, T, 128]  values
+ *   mask         [B, 1,  T, mask_ld] additive bf16 mask (entries j < T used),
+ *                or NULL for the implicit causal mask (key j allowed iff j <= i).
+ *                A non-NULL mask is applied exactly as given, with no extra
+ *                causal term; -inf entries exclude a key. A row with no
+ *                allowed key produces zeros.
+ *   mask_ld      row stride of mask in elements (>= T); ignored when mask is
+ *                NULL. Rows are read with 16-byte loads when mask is 16-byte
+ *                aligned and mask_ld % 8 == 0, with 2-byte loads otherwise.
+ *   B, T         batch (1..65535) and sequence length (1..8388480); keys = queries = T
+ *   softmax_scale  multiplies Q.K^T before the mask is added (finite)
+ *   workspace    device scratch of mla_attn_prefill_workspace_bytes(B,T,mask!=NULL)
+ *                bytes; may be NULL when mask is NULL. Contents on entry are
+ *                ignored; the call must not overlap another call using it.
+ *   out          [B, T, 8192]: out[b,i,h*128+e], bf16
+ */
+mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                              const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                              const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                              int T, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
+
+/*
+ * Output projection, nn.Linear(8192 -> 7168, bias=False)
+ * (page "Kimi K2 · Mix and project", excerpt modeling_deepseek.py 848-852 and
+ * the page's parameter table: 8,192 x 7,168 = 58,720,256 weights):
+ *
+ *   attn  [M, 8192] bf16 (merged heads, row = token)
+ *   W_o   [7168, 8192] bf16 (out_features, in_features)
+ *   M     rows, 1 .. 2^31 - 129
+ *   out   [M, 7168] bf16 = attn . W_o^T, fp32 accumulation, rounded once
+ */
+mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, mla_bf16* out,
+                        mla_stream_t stream);
+
+/*
+ * Workspace bytes mla_attn_oproj needs: B*T*8192*2 bytes for the merged
+ * attention output, rounded up to 256, plus the mask-class bytes when
+ * has_mask != 0. Returns 0 for B < 1 or T < 1.
+ */
+size_t mla_attn_oproj_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * Attention followed by o_proj: the whole path of the page
+ * "Kimi K2 · Mix and project" from the per-head inputs to Delta_attn.
+ * Arguments as in mla_attn_prefill and mla_o_proj; the merged attention output
+ * lives in `workspace` (mla_attn_oproj_workspace_bytes bytes, required), and
+ *   out   [B, T, 7168] bf16.
+ */
+mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                            const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                            const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                            int T, float softmax_scale, const mla_bf16* W_o, void* workspace,
+                            size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns MLA_ERR_TIMEOUT if any kernel of this library gave
+ * up on a bounded wait since the last call, MLA_ERR_CUDA if the stream
+ * reports an error, else MLA_OK. If `detail` is not NULL it receives the raw
+ * status word (kernel id << 8 | wait site, timeout flag in bit 16).
+ */
+mla_status_t mla_device_status(mla_stream_t stream, uint32_t* detail);
+
+/* Static, human-readable name of a status code. */
+const char* mla_status_string(mla_status_t status);
+
+/* MLA_ABI_VERSION of the loaded library. */
+int mla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

@@ -2,16 +2,10 @@
 
 The compute lives in hand-written CUDA kernels behind a C ABI
 (``include/mla.h``, built into ``libmla_b200.so`` next to this file);
-``binding`` is a thin ctypes layer over it. Importing the package does not
-load the library; the first call does, and fails loudly if it is missing.
+``mla_causal_attention_attn_b200.binding`` is a thin ctypes layer over it.
+Importing the package does not load the library; the first call does, and
+fails loudly if it is missing.
 """
 from . import inputs  # noqa: F401  (seeded synthetic inputs, no arithmetic)
 
-__all__ = ["inputs", "binding"]
-
-
-def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    raise AttributeError(name)
+__all__ = ["inputs"]

@@ -1,0 +1,204 @@
+"""ctypes binding of ``libmla_b200.so`` (declared in ``include/mla.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI. PyTorch provides device memory and streams. There
+is no fallback: if the library is missing or fails to load, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import inputs as _inputs
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmla_b200.so")
+
+H = _inputs.H
+DN, DR, DV = _inputs.DN, _inputs.DR, _inputs.DV
+D_MODEL = _inputs.D_MODEL
+K_OPROJ = _inputs.K_OPROJ
+
+STATUS = {
+    0: "MLA_OK",
+    -1: "MLA_ERR_INVALID_ARG",
+    -2: "MLA_ERR_SHAPE",
+    -3: "MLA_ERR_MISALIGNED",
+    -4: "MLA_ERR_UNSUPPORTED_DEVICE",
+    -5: "MLA_ERR_WORKSPACE",
+    -6: "MLA_ERR_CUDA",
+    -7: "MLA_ERR_TIMEOUT",
+}
+MLA_OK = 0
+
+# Every symbol include/mla.h declares, with its ctypes signature.
+_VP = ctypes.c_void_p
+_SIGNATURES = {
+    "mla_attn_prefill_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_prefill": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_float, _VP, ctypes.c_size_t, _VP,
+                                        _VP]),
+    "mla_o_proj": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, _VP, _VP]),
+    "mla_attn_oproj_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_oproj": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_float, _VP, _VP, ctypes.c_size_t, _VP,
+                                      _VP]),
+    "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
+    "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_abi_version": (ctypes.c_int, []),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MLAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the library (once). Raises if it is missing."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or LIB_PATH
+            if not os.path.exists(p):
+                raise RuntimeError(
+                    f"{p} is missing: build it with `python -m mla_causal_attention_attn_b200.build`")
+            lib = ctypes.CDLL(p)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != MLA_OK:
+        raise MLAError(fn, status)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def _req(t, shape, name):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bf16, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def attn_prefill_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_prefill_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def attn_oproj_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_oproj_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def _mask_ld(mask, B, T):
+    """Row stride of a [B,1,T,T] mask view whose rows are ``ld`` elements apart
+    and whose batches are ``T*ld`` apart (a dense [B,1,T,ld] buffer)."""
+    if mask is None:
+        return 0
+    if mask.dtype != torch.bfloat16 or not mask.is_cuda:
+        raise TypeError("mask must be a bf16 CUDA tensor")
+    if mask.dim() != 4 or tuple(mask.shape) != (B, 1, T, T):
+        raise ValueError(f"mask must be [B,1,T,T] = {(B, 1, T, T)}, got {tuple(mask.shape)}")
+    ld = int(mask.stride(2)) if T > 1 else max(int(mask.stride(2)), T)
+    if mask.stride(3) != 1 or ld < T or (B > 1 and mask.stride(0) != T * ld):
+        raise ValueError("mask must be a view of a dense [B,1,T,ld] buffer")
+    return ld
+
+
+def attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask=None, softmax_scale=None, out=None,
+                 workspace=None, stream=None):
+    """Merged-head attention output [B, T, 8192] (bf16) via ``mla_attn_prefill``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, K_OPROJ), "out")
+    need = attn_prefill_workspace_bytes(B, T, mask is not None)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.mla_attn_prefill(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                              _ptr(mask), mask_ld, B, T, scale, _ptr(workspace), ws_bytes,
+                              _ptr(out), _stream_handle(stream))
+    _check("mla_attn_prefill", st)
+    return out
+
+
+def o_proj(attn, W_o, out=None, stream=None):
+    """``attn [M, 8192] . W_o^T`` -> [M, 7168] (bf16) via ``mla_o_proj``."""
+    lib = load()
+    a2 = attn.reshape(-1, K_OPROJ)
+    M = a2.shape[0]
+    _req(a2, (M, K_OPROJ), "attn")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    if out is None:
+        out = torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=attn.device)
+    _req(out.view(-1, D_MODEL), (M, D_MODEL), "out")
+    st = lib.mla_o_proj(_ptr(a2), _ptr(W_o), M, _ptr(out), _stream_handle(stream))
+    _check("mla_o_proj", st)
+    return out
+
+
+def attn_oproj(q_nope, q_pe, k_nope, k_pe, v, W_o, mask=None, softmax_scale=None, out=None,
+               workspace=None, stream=None):
+    """Whole path: attention then o_proj, [B, T, 7168] bf16, via ``mla_attn_oproj``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    need = attn_oproj_workspace_bytes(B, T, mask is not None)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.mla_attn_oproj(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                            _ptr(mask), mask_ld, B, T, scale, _ptr(W_o), _ptr(workspace),
+                            ws_bytes, _ptr(out), _stream_handle(stream))
+    _check("mla_attn_oproj", st)
+    return out
+
+
+def device_status(stream=None):
+    """Synchronise the stream; return (status, raw status word)."""
+    lib = load()
+    detail = ctypes.c_uint32(0)
+    st = lib.mla_device_status(_stream_handle(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)

@@ -1,0 +1,29 @@
+// host_util.h -- host-side helpers shared by the launchers: TMA tensor-map
+// encoding through the driver entry point, per-device SM count cache and
+// kernel-attribute setup.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace mla {
+
+// Encode a row-major bf16 tensor of `rank` dims (dims[0] innermost, in
+// elements; strides_bytes[i] is the byte stride of dim i+1) as a TMA tiled map
+// with 128-byte swizzle and zero fill out of bounds. Returns false when the
+// driver rejects the map.
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
+// Number of SMs of the current device (cached per device ordinal).
+int device_sm_count();
+
+// Compute capability major*10+minor of the current device (cached).
+int device_cc();
+
+// Sets the max-dynamic-shared-memory attribute of `func` once per device
+// (one bit of *done_mask per device ordinal).
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);
+
+}  // namespace mla

@@ -1,0 +1,205 @@
+// mla_abi.cu -- the extern "C" entry points declared in include/mla.h:
+// argument validation, workspace carving, then kernel launches on the
+// caller's stream.
+#include <cmath>
+#include <cstdlib>
+
+#include "../../include/mla.h"
+#include "attn_prefill.h"
+#include "host_util.h"
+#include "oproj_gemm.h"
+#include "sm100.cuh"
+
+namespace mla {
+
+// The library's device status word (one per device that loads the library).
+__device__ unsigned int g_device_error = 0;
+
+namespace {
+
+// Device address of g_device_error for the current device, fetched once per
+// device; null if the runtime cannot provide it.
+unsigned int* device_error_word() {
+  constexpr int kMaxDev = 64;
+  static unsigned int* addr[kMaxDev] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  unsigned int* p = __atomic_load_n(&addr[dev], __ATOMIC_ACQUIRE);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
+    p = static_cast<unsigned int*>(a);
+    __atomic_store_n(&addr[dev], p, __ATOMIC_RELEASE);
+  }
+  return p;
+}
+
+constexpr int kMaxB = 65535;
+constexpr int kMaxT = 65535 * 128;
+constexpr int64_t kMaxM = (int64_t(1) << 31) - 129;
+
+unsigned long long wait_limit_ns() {
+  // MLA_WAIT_LIMIT_NS overrides the per-wait limit (read once).
+  static const unsigned long long v = [] {
+    const char* s = std::getenv("MLA_WAIT_LIMIT_NS");
+    if (s && *s) {
+      char* end = nullptr;
+      unsigned long long x = std::strtoull(s, &end, 10);
+      if (end && *end == '\0' && x > 0) return x;
+    }
+    return kDefaultWaitLimitNs;
+  }();
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+mla_status_t check_device() {
+  const int cc = device_cc();
+  if (cc == 0) return MLA_ERR_CUDA;
+  if (cc != 100) return MLA_ERR_UNSUPPORTED_DEVICE;
+  if (!device_error_word()) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+mla_status_t check_attn_args(const void* q_nope, const void* q_pe, const void* k_nope,
+                             const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
+                             int B, int T, float softmax_scale, const void* out) {
+  if (!q_nope || !q_pe || !k_nope || !k_pe || !v || !out) return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return MLA_ERR_SHAPE;
+  if (mask && mask_ld < T) return MLA_ERR_SHAPE;
+  if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(k_nope) || !aligned16(k_pe) ||
+      !aligned16(v) || !aligned16(out))
+    return MLA_ERR_MISALIGNED;
+  if (mask && (reinterpret_cast<uintptr_t>(mask) & 1u) != 0) return MLA_ERR_MISALIGNED;
+  return MLA_OK;
+}
+
+mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
+                           const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
+                           int B, int T, float softmax_scale, void* cls, void* out,
+                           cudaStream_t stream) {
+  if (mask) {
+    mla_status_t s = from_cuda(launch_mask_classify(mask, mask_ld, B, T, cls, stream));
+    if (s != MLA_OK) return s;
+  }
+  return from_cuda(launch_attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld,
+                                       mask ? cls : nullptr, B, T, softmax_scale, out,
+                                       wait_limit_ns(), device_error_word(), stream));
+}
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+extern "C" {
+
+size_t mla_attn_prefill_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  return has_mask ? attn_class_bytes(B, T) : 0;
+}
+
+mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                              const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                              const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                              int T, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if (mask) {
+    if (!workspace || workspace_bytes < attn_class_bytes(B, T)) return MLA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  }
+  s = check_device();
+  if (s != MLA_OK) return s;
+  return run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale,
+                       workspace, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, mla_bf16* out,
+                        mla_stream_t stream) {
+  if (!attn || !W_o || !out) return MLA_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
+  if (!aligned16(attn) || !aligned16(W_o) || !aligned16(out)) return MLA_ERR_MISALIGNED;
+  mla_status_t s = check_device();
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(attn, W_o, out, M, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, device_error_word(),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_attn_oproj_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  size_t bytes = round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
+  if (has_mask) bytes += round_up(attn_class_bytes(B, T), 256);
+  return bytes;
+}
+
+mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                            const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                            const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                            int T, float softmax_scale, const mla_bf16* W_o, void* workspace,
+                            size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if (!W_o) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_o)) return MLA_ERR_MISALIGNED;
+  if (int64_t(B) * int64_t(T) > kMaxM) return MLA_ERR_SHAPE;
+  const size_t need = mla_attn_oproj_workspace_bytes(B, T, mask != nullptr);
+  if (!workspace || workspace_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t attn_bytes = round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
+  void* attn = ws;
+  void* cls = mask ? ws + attn_bytes : nullptr;
+  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale, cls,
+                    attn, st);
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, device_error_word(),
+                                     st));
+}
+
+mla_status_t mla_device_status(mla_stream_t stream, uint32_t* detail) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return MLA_ERR_CUDA;
+  }
+  if (detail) *detail = word;
+  return (word & kErrTimeoutFlag) ? MLA_ERR_TIMEOUT : MLA_OK;
+}
+
+const char* mla_status_string(mla_status_t status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_SHAPE: return "MLA_ERR_SHAPE";
+    case MLA_ERR_MISALIGNED: return "MLA_ERR_MISALIGNED";
+    case MLA_ERR_UNSUPPORTED_DEVICE: return "MLA_ERR_UNSUPPORTED_DEVICE";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,294 @@
+// oproj_gemm.cu -- the output projection C[M, N] = A[M, K] . W[N, K]^T in bf16
+// with fp32 accumulation (page "Kimi K2 · Mix and project": o_proj is
+// nn.Linear(64*128 -> 7168, bias=False) applied to the merged heads; the
+// page's parameter table gives W 8,192 x 7,168).
+//
+// Design (sm_100a):
+//   * persistent CTAs, one per SM, walking 128 x BN output tiles in a
+//     GROUP_M-swizzled order so concurrently running CTAs share A and W tiles
+//     in L2;
+//   * warp 0 issues TMA loads of 128x64 A and BNx64 W tiles (128-byte
+//     swizzle) into a STAGES-deep shared-memory ring;
+//   * warp 1 allocates tensor memory and one elected thread issues
+//     tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators;
+//   * warps 2..5 drain the finished accumulator (tcgen05.ld), convert to bf16
+//     and store, while the MMA warp already fills the other accumulator.
+#include "oproj_gemm.h"
+#include "host_util.h"
+#include "sm100.cuh"
+
+namespace mla {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGroupM = 16;
+constexpr int kThreads = 192;
+
+__device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
+                                                 int& nb) {
+  const int group_tiles = kGroupM * n_tiles;
+  const int group = tile / group_tiles;
+  const int first_m = group * kGroupM;
+  const int gm = min(kGroupM, m_tiles - first_m);
+  const int in_group = tile - group * group_tiles;
+  mb = first_m + in_group % gm;
+  nb = in_group / gm;
+}
+
+template <int BN, int STAGES>
+struct GemmCfg {
+  static constexpr uint32_t kABytes = kBM * kBK * 2;
+  static constexpr uint32_t kBBytes = BN * kBK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+  static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+  static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                "TMEM columns must be a power of two in [32, 512]");
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    oproj_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, __nv_bfloat16* __restrict__ C,
+                      int M, int N, int K, unsigned long long wait_limit_ns,
+                      unsigned int* err_word) {
+  using Cfg = GemmCfg<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full_bar[STAGES];
+  __shared__ uint64_t empty_bar[STAGES];
+  __shared__ uint64_t acc_full[2];
+  __shared__ uint64_t acc_empty[2];
+  __shared__ uint64_t drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  // 1024-byte aligned start of the stage ring (128B-swizzle atoms).
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m_tiles = (M + kBM - 1) / kBM;
+  const int n_tiles = N / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int k_blocks = K / kBK;
+
+  WaitCtl ctl{&abort_flag, wait_limit_ns, kErrKernelOproj, err_word};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        gemm_tile_coords(tile, m_tiles, n_tiles, mb, nb);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, ctl, 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
+          uint8_t* sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBK, mb * kBM);
+          tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBK, nb * BN);
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA's memory goes away.
+        int zero = 0;
+        WaitCtl drain{&zero, wait_limit_ns, kErrKernelOproj, err_word};
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) mbar_wait(&full_bar[s], (issued_par >> s) & 1u, drain, 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t acc_par = (local >> 1) & 1;
+        if (!mbar_wait(&acc_empty[buf], acc_par ^ 1u, ctl, 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(buf * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, ctl, 4)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + size_t(stage) * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          mma_commit(&empty_bar[stage]);  // frees the stage once these MMAs finish
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit(&acc_full[buf]);
+      }
+      if (!ok && issued_any) {
+        // Wait for the MMAs in flight before the tensor memory is released.
+        mma_commit(&drain_bar);
+        int zero = 0;
+        WaitCtl drain{&zero, wait_limit_ns, kErrKernelOproj, err_word};
+        mbar_wait(&drain_bar, 0, drain, 5);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row_in_tile = quad * 32 + lane;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      int mb, nb;
+      gemm_tile_coords(tile, m_tiles, n_tiles, mb, nb);
+      const int buf = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      if (!mbar_wait_warp(&acc_full[buf], acc_par, ctl, 6)) break;
+      tc_fence_after();
+      const int row = mb * kBM + row_in_tile;
+      __nv_bfloat16* crow = C + size_t(row) * size_t(N) + size_t(nb) * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_addr(tmem_base, quad * 32, buf * BN + c * 32), r);
+        tmem_ld_wait();
+        reg_fence(r);
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        if (row < M) {
+          uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, int M, int N,
+                      int K, int num_sms, unsigned long long wait_limit_ns,
+                      unsigned int* err_word, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN, STAGES>;
+  CUtensorMap tmB;
+  const uint64_t dims[2] = {uint64_t(K), uint64_t(N)};
+  const uint64_t strides[1] = {uint64_t(K) * 2};
+  const uint32_t box[2] = {kBK, BN};
+  if (!encode_tmap_bf16(&tmB, W, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
+  auto kern = oproj_gemm_kernel<BN, STAGES>;
+  static unsigned attr_done = 0;  // one bit per device ordinal
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
+                                   &attr_done);
+  if (e != cudaSuccess) return e;
+  const int m_tiles = (M + kBM - 1) / kBM;
+  const int num_tiles = m_tiles * (N / BN);
+  const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+  kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(tmA, tmB, C, M, N, K, wait_limit_ns,
+                                                   err_word);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int oproj_pick_bn(int64_t M, int N, int num_sms) {
+  const int64_t m_tiles = (M + kBM - 1) / kBM;
+  if (m_tiles * (N / 256) >= num_sms) return 256;
+  if (m_tiles * (N / 128) >= num_sms) return 128;
+  return 64;
+}
+
+cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
+                              int num_sms, unsigned long long wait_limit_ns, int force_bn,
+                              unsigned int* err_word, cudaStream_t stream) {
+  if (M <= 0 || N % 256 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
+    return cudaErrorInvalidValue;
+  CUtensorMap tmA;
+  const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
+  const uint64_t strides[1] = {uint64_t(K) * 2};
+  const uint32_t box[2] = {kBK, kBM};
+  if (!encode_tmap_bf16(&tmA, A, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
+  const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
+  auto* Cb = static_cast<__nv_bfloat16*>(C);
+  switch (bn) {
+    case 256:
+      return launch_bn<256, 4>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+                                 stream);
+    case 128:
+      return launch_bn<128, 6>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+                                 stream);
+    case 64:
+      return launch_bn<64, 8>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+                                 stream);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace mla

@@ -131,8 +131,10 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
 #pragma omp for schedule(dynamic, 4)
         for (int64_t w = 0; w < work; ++w) {
             if (!s || !qv || !acc) continue;
-            const int64_t r = w / H;
-            const int h = (int)(w % H);
+            /* consecutive work items share a head, so the threads stream the
+               same keys and values */
+            const int h = (int)(w / nrows);
+            const int64_t r = w % nrows;
             const int64_t b = row_b[r];
             const int64_t i = row_i[r];
             const int64_t bh = b * H + h;

@@ -1,0 +1,137 @@
+"""Host-only checks of the C ABI (no GPU needed).
+
+The library must load, export every function include/mla.h declares, and
+reject bad arguments with the documented status codes before it touches the
+device. Fake non-null device addresses are used: argument validation runs
+before any CUDA call, so they are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from mla_causal_attention_attn_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+OK, INVALID, SHAPE, MISALIGNED, UNSUPPORTED, WORKSPACE, CUDA, TIMEOUT = 0, -1, -2, -3, -4, -5, -6, -7
+A = 0x7f0000000000  # a 16-byte aligned fake device address, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("mla_attn_prefill", "mla_o_proj", "mla_attn_oproj"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding._SIGNATURES), "binding signatures drift from the header"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.mla_abi_version() == 1
+    for code, name in binding.STATUS.items():
+        assert lib.mla_status_string(code).decode() == name
+    assert lib.mla_status_string(12345).decode() == "MLA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    assert lib.mla_attn_prefill_workspace_bytes(1, 4096, 0) == 0
+    assert lib.mla_attn_prefill_workspace_bytes(8, 4096, 1) == 8 * 32 * 32
+    assert lib.mla_attn_prefill_workspace_bytes(2, 129, 1) == 2 * 2 * 2
+    assert lib.mla_attn_prefill_workspace_bytes(0, 10, 1) == 0
+    attn = 1 * 4096 * 8192 * 2
+    assert lib.mla_attn_oproj_workspace_bytes(1, 4096, 0) == attn
+    assert lib.mla_attn_oproj_workspace_bytes(8, 4096, 1) == 8 * 4096 * 8192 * 2 + 8 * 32 * 32
+    assert lib.mla_attn_oproj_workspace_bytes(1, 3, 0) == 49152  # 3*8192*2 rounded to 256
+    assert lib.mla_attn_oproj_workspace_bytes(-1, 3, 0) == 0
+
+
+def prefill(lib, q=A, qp=A, k=A, kp=A, v=A, mask=None, ld=0, B=1, T=64, scale=0.07,
+            ws=None, ws_bytes=0, out=A):
+    return lib.mla_attn_prefill(q, qp, k, kp, v, mask, ld, B, T, scale, ws, ws_bytes, out, None)
+
+
+def fused(lib, q=A, qp=A, k=A, kp=A, v=A, mask=None, ld=0, B=1, T=64, scale=0.07, W=A,
+          ws=A, ws_bytes=1 << 40, out=A):
+    return lib.mla_attn_oproj(q, qp, k, kp, v, mask, ld, B, T, scale, W, ws, ws_bytes, out, None)
+
+
+def test_prefill_argument_errors(lib):
+    assert prefill(lib, q=None) == INVALID
+    assert prefill(lib, kp=None) == INVALID
+    assert prefill(lib, out=None) == INVALID
+    assert prefill(lib, scale=float("nan")) == INVALID
+    assert prefill(lib, scale=float("inf")) == INVALID
+    assert prefill(lib, B=0) == SHAPE
+    assert prefill(lib, T=0) == SHAPE
+    assert prefill(lib, T=-5) == SHAPE
+    assert prefill(lib, B=65536) == SHAPE
+    assert prefill(lib, T=65535 * 128 + 1) == SHAPE
+    assert prefill(lib, mask=A, ld=32, T=64, ws=A, ws_bytes=64) == SHAPE  # ld < T
+    assert prefill(lib, q=A + 8) == MISALIGNED
+    assert prefill(lib, v=A + 2) == MISALIGNED
+    assert prefill(lib, out=A + 4) == MISALIGNED
+    assert prefill(lib, mask=A + 1, ld=64, ws=A, ws_bytes=64) == MISALIGNED  # odd address
+    assert prefill(lib, mask=A, ld=64) == WORKSPACE                       # none given
+    assert prefill(lib, mask=A, ld=304, B=2, T=300, ws=A, ws_bytes=17) == WORKSPACE  # need 18
+
+
+def test_oproj_argument_errors(lib):
+    assert lib.mla_o_proj(None, A, 4, A, None) == INVALID
+    assert lib.mla_o_proj(A, None, 4, A, None) == INVALID
+    assert lib.mla_o_proj(A, A, 4, None, None) == INVALID
+    assert lib.mla_o_proj(A, A, 0, A, None) == SHAPE
+    assert lib.mla_o_proj(A, A, -1, A, None) == SHAPE
+    assert lib.mla_o_proj(A, A, 1 << 31, A, None) == SHAPE
+    assert lib.mla_o_proj(A + 2, A, 4, A, None) == MISALIGNED
+    assert lib.mla_o_proj(A, A + 8, 4, A, None) == MISALIGNED
+
+
+def test_fused_argument_errors(lib):
+    assert fused(lib, W=None) == INVALID
+    assert fused(lib, q=None) == INVALID
+    assert fused(lib, B=0) == SHAPE
+    assert fused(lib, W=A + 2) == MISALIGNED
+    assert fused(lib, ws=None) == WORKSPACE
+    assert fused(lib, ws_bytes=64 * 8192 * 2 - 1) == WORKSPACE
+    assert fused(lib, ws=A + 8) == MISALIGNED
+    assert fused(lib, mask=A, ld=64, ws_bytes=64 * 8192 * 2) == WORKSPACE  # class bytes missing
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path only")
+def test_valid_call_without_device_reports_cuda_error(lib):
+    """With no usable device a well-formed call fails cleanly (MLA_ERR_CUDA)
+    instead of launching anything."""
+    assert prefill(lib) in (CUDA, UNSUPPORTED)
+    assert lib.mla_o_proj(A, A, 4, A, None) in (CUDA, UNSUPPORTED)
+
+
+def test_binding_refuses_missing_library(tmp_path):
+    with pytest.raises(RuntimeError):
+        old = binding._lib
+        try:
+            binding._lib = None
+            binding.load(str(tmp_path / "nope.so"))
+        finally:
+            binding._lib = old

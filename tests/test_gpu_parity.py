@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small shapes are compared element by element on every row; they span several
+128-row / 128-key tiles and ragged tails. The five full-size workloads are
+compared on sampled rows (the oracle evaluates any row on its own), launched
+exactly as the benchmark launches them.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_causal_attention_attn_b200 import binding, inputs
+from parity import assert_parity, metrics, sample_rows, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def to_dev(d, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def oracle_attn(d, rows=None):
+    return oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], d["mask"],
+                            d["softmax_scale"], rows=rows)
+
+
+def gpu_attn(g, stream=None):
+    return binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                mask=g["mask"], softmax_scale=g["softmax_scale"], stream=stream)
+
+
+def gpu_full(g):
+    return binding.attn_oproj(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"], g["W_o"],
+                              mask=g["mask"], softmax_scale=g["softmax_scale"])
+
+
+def check_status():
+    st, word = binding.device_status()
+    assert st == 0, f"device status {binding.STATUS.get(st, st)} word={word:#x}"
+
+
+# ------------------------------------------------------------------ o_proj
+@pytest.mark.parametrize("M", [1, 64, 129, 300, 1000])
+def test_oproj_all_rows(cuda_device, M):
+    """mla_o_proj on every row; M picks 64-, 128- and 256-wide tiles."""
+    g = torch.Generator().manual_seed(M)
+    attn = torch.randn(M, inputs.K_OPROJ, generator=g).to(torch.bfloat16)
+    W = (torch.randn(inputs.D_MODEL, inputs.K_OPROJ, generator=g) * 0.02).to(torch.bfloat16)
+    out = binding.o_proj(attn.to(cuda_device), W.to(cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref = oracle.oproj_rows(oracle.bf16_to_f64(attn), W)
+    assert_parity(to_f64(out), ref, f"o_proj M={M}")
+
+
+def test_oproj_large_sampled(cuda_device):
+    M = 4096 + 77
+    g = torch.Generator().manual_seed(5)
+    attn = torch.randn(M, inputs.K_OPROJ, generator=g).to(torch.bfloat16)
+    W = (torch.randn(inputs.D_MODEL, inputs.K_OPROJ, generator=g) * 0.02).to(torch.bfloat16)
+    out = binding.o_proj(attn.to(cuda_device), W.to(cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    rows = sorted(set([0, 1, 127, 128, 129, M - 1, M - 2, M - 78, M - 77]
+                      + list(np.random.default_rng(0).integers(0, M, 100))))
+    ref = oracle.oproj_rows(oracle.bf16_to_f64(attn[rows]), W)
+    assert_parity(to_f64(out[rows]), ref, "o_proj M=4173 sampled")
+
+
+# ------------------------------------------------------------------ attention
+CAUSAL_SHAPES = [(1, 1), (1, 2), (2, 63), (1, 64), (1, 65), (1, 127), (1, 128), (2, 129),
+                 (1, 255), (1, 257), (3, 300), (1, 512)]
+
+
+@pytest.mark.parametrize("B,T", CAUSAL_SHAPES)
+def test_attn_causal_all_rows(cuda_device, B, T):
+    d = inputs.make_inputs(B, T, seed=T * 10 + B, with_weight=False)
+    out = gpu_attn(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, fm = oracle_attn(d)
+    assert not fm.any()
+    assert_parity(to_f64(out).reshape(B * T, -1), ref, f"attn causal B={B} T={T}")
+
+
+@pytest.mark.parametrize("B,T,min_valid", [(3, 300, 1), (2, 256, 100), (2, 129, 1), (1, 64, 7)])
+def test_attn_keypad_mask_all_rows(cuda_device, B, T, min_valid):
+    d = inputs.make_inputs(B, T, seed=B * 1000 + T, key_padding=True, min_valid=min_valid,
+                           with_weight=False)
+    out = gpu_attn(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, fm = oracle_attn(d)
+    assert not fm.any()
+    assert_parity(to_f64(out).reshape(B * T, -1), ref, f"attn keypad B={B} T={T}")
+
+
+def test_attn_general_additive_mask_and_fully_masked_rows(cuda_device):
+    """Finite non-zero mask values, -inf holes, a mask row stride larger than
+    T, and rows with no allowed key (written as zeros)."""
+    B, T, ld = 2, 200, 208
+    d = inputs.make_inputs(B, T, seed=77, with_weight=False)
+    g = torch.Generator().manual_seed(3)
+    m = torch.randn(B, 1, T, ld, generator=g) * 2.0
+    holes = torch.rand(B, 1, T, ld, generator=g) < 0.3
+    m[holes] = float("-inf")
+    m[0, 0, 5, :] = float("-inf")          # fully masked rows
+    m[1, 0, 150, :] = float("-inf")
+    m[1, 0, 0:128, 128:] = float("-inf")   # a whole tile skipped
+    m[0, 0, 128:, 128:] = 0.0              # a whole all-zero tile
+    mask = m.to(torch.bfloat16)
+    d["mask"] = mask[..., :T]
+    ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                               d["mask"].contiguous(), d["softmax_scale"])
+    gd = to_dev(d, cuda_device)
+    gd["mask"] = mask.to(cuda_device)[..., :T]  # strided view, row stride ld
+    out = gpu_attn(gd)
+    torch.cuda.synchronize()
+    check_status()
+    got = to_f64(out).reshape(B * T, -1)
+    rows_fm = fm.any(axis=1)
+    assert rows_fm[5] and rows_fm[T + 150]
+    assert np.all(got[rows_fm] == 0.0)
+    assert_parity(got[~rows_fm], ref[~rows_fm], "attn general mask")
+
+
+def test_attn_causal_future_invariance(cuda_device):
+    """Rows <= t are bit-identical after changing keys/values at positions > t."""
+    B, T, t = 1, 300, 140
+    d = inputs.make_inputs(B, T, seed=9, with_weight=False)
+    a = gpu_attn(to_dev(d, cuda_device)).clone()
+    d2 = dict(d)
+    for k in ("k_nope", "k_pe", "v"):
+        x = d[k].clone()
+        x[:, :, t + 1:] = (x[:, :, t + 1:].float() * -3.0 + 1.0).to(torch.bfloat16)
+        d2[k] = x
+    b2 = gpu_attn(to_dev(d2, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    assert torch.equal(a[:, : t + 1], b2[:, : t + 1])
+    assert not torch.equal(a[:, t + 1:], b2[:, t + 1:])
+
+
+def test_attn_on_side_stream(cuda_device):
+    d = inputs.make_inputs(1, 200, seed=4, with_weight=False)
+    s = torch.cuda.Stream()
+    gd = to_dev(d, cuda_device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        out = gpu_attn(gd, stream=s)
+    s.synchronize()
+    ref, _ = oracle_attn(d)
+    assert_parity(to_f64(out).reshape(200, -1), ref, "side stream")
+
+
+# ------------------------------------------------------------------ whole path
+def test_fused_small_all_rows(cuda_device):
+    """B=1, T=64 causal (the small workload), every output element."""
+    d = inputs.make_workload(inputs.WORKLOADS["b1_t64_causal"])
+    out = gpu_full(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, fm = oracle.attn_oproj_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                                     None, d["softmax_scale"], d["W_o"])
+    assert not fm.any()
+    m = assert_parity(to_f64(out).reshape(64, -1), ref, "fused b1_t64")
+    print(m)
+
+
+def test_fused_ragged_all_rows(cuda_device):
+    d = inputs.make_inputs(2, 200, seed=21)
+    out = gpu_full(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, _ = oracle.attn_oproj_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                                    None, d["softmax_scale"], d["W_o"])
+    assert_parity(to_f64(out).reshape(400, -1), ref, "fused B=2 T=200")
+
+
+FULL = ["b1_t4096_causal", "b16_t1024_causal", "b8_t4096_keypad_mask", "b1_t32768_causal_qx2"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_fused_full_size_sampled_rows(cuda_device, name):
+    w = inputs.WORKLOADS[name]
+    d = inputs.make_workload(w)
+    n_random = 300 if w.T >= 32768 else 600
+    rows = sample_rows(w.B, w.T, n_random, seed=1, valid_len=d["valid_len"])
+    gd = to_dev(d, cuda_device)
+    out = gpu_full(gd)
+    torch.cuda.synchronize()
+    check_status()
+    got = to_f64(out[[r[0] for r in rows], [r[1] for r in rows]])
+    del gd, out
+    ref, fm = oracle.attn_oproj_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                                     d["mask"], d["softmax_scale"], d["W_o"], rows=rows)
+    assert not fm.any()
+    m = assert_parity(got, ref, f"{name} ({len(rows)} rows)")
+    print(name, len(rows), m)
