@@ -9,20 +9,27 @@
 //   with k_pe one [B,1,T,64] tensor shared by all heads and M either the
 //   implicit causal mask (mask == NULL) or an explicit additive [B,1,T,T] mask.
 //
-// One CTA computes one (b, h, 128-row query tile); the longest causal tiles
-// are scheduled first. Roles:
-//   warp 0      TMA producer: the Q tile (nope + rope, 48 KB) once, then per
-//               128-key tile the K tile (k_nope + the shared k_pe, 48 KB) and
-//               the V tile (32 KB) into 2-deep rings;
-//   warp 1      tensor-memory owner and MMA issuer:
-//                 S_j = Q K_j^T     128x128, K = 128 (nope) + 64 (rope), SS
-//                 O  += P_j V_j     128x128, K = 128 keys, P from TMEM (TS)
-//               S is double-buffered so S_{j+1} runs while row softmax j does;
-//   warps 2..5  one thread per query row: read S_j from TMEM, scale, mask,
-//               online max (rescaling O only when the max grows by more than
-//               2^8), exponentials, row sum, write P_j as bf16 back into the S
-//               buffer, and at the end O / l -> bf16 -> out[b, i, h*128 ..].
-// Tensor memory: S0 cols [0,128), S1 [128,256), O [256,384).
+// One CTA computes two 128-row query tiles (2p, 2p+1) of one (b, h), so that
+// every K/V tile brought into shared memory serves 256 query rows and the
+// softmax of one query tile overlaps the tensor-core work of the other.
+// Roles (384 threads = three warpgroups):
+//   warp 0       TMA producer: both Q tiles (nope + rope, 48 KB each) once,
+//                then for every visited 128-key tile five 16 KB blocks
+//                (k_nope lo/hi, the shared k_pe, v lo/hi) into an 8-block ring;
+//   warp 1       tensor-memory owner and MMA issuer. Per key tile j, in order:
+//                  O0 += P0_{j-1} V_{j-1},  S0 = Q0 K_j^T,
+//                  O1 += P1_{j-1} V_{j-1},  S1 = Q1 K_j^T
+//                (S: 128x128, K = 128 nope + 64 rope, both operands in shared
+//                memory; PV: 128x128, K = 128 keys, P read from tensor memory).
+//                Because PV_{j-1} of a tile is issued before its S_j, the
+//                commit that announces S_j also guarantees O holds PV_{j-1};
+//   warps 2, 3   idle;
+//   warps 4..7   softmax of query tile 0, one thread per row (TMEM lane);
+//   warps 8..11  softmax of query tile 1. Each reads S, scales, masks, keeps a
+//                running max (rescaling O only when the max grows by more than
+//                2^8), exponentiates, sums, writes P as bf16 over the first 64
+//                columns of its S buffer, and at the end O / l -> bf16 -> out.
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 #include "attn_prefill.h"
 #include "host_util.h"
 #include "sm100.cuh"
@@ -31,29 +38,33 @@ namespace mla {
 
 namespace {
 
-constexpr int kBQ = 128;     // query rows per CTA
+constexpr int kBQ = 128;     // query rows per tile
 constexpr int kBKV = 128;    // keys per tile
 constexpr int kDN = 128;     // qk_nope_head_dim
 constexpr int kDR = 64;      // qk_rope_head_dim
 constexpr int kDV = 128;     // v_head_dim
 constexpr int kH = 64;       // heads
-constexpr int kNSK = 2;      // K ring depth
-constexpr int kNSV = 2;      // V ring depth
-constexpr int kThreads = 192;
+constexpr int kHeadGroup = 8;  // heads whose CTAs are scheduled together (L2 reuse of K/V)
+constexpr int kRing = 8;     // 16 KB blocks in the K/V ring
+constexpr int kBlocksPerTile = 5;
+constexpr int kThreads = 384;
+// ptxas budgets 168 registers a thread for 384 threads; setmaxnreg moves
+// them: 128 x 88 (warpgroup 0) + 256 x 208 (softmax) = 384 x 168.
+constexpr uint32_t kRegsControl = 88;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * 168, "register split");
+constexpr int kBarTeardown = 1;  // named barrier for the final hand-off
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 
-constexpr uint32_t kBlock = kBQ * 64 * 2;      // one 128 x 64 bf16 swizzled block: 16 KB
-constexpr uint32_t kQBytes = 3 * kBlock;       // nope lo, nope hi, rope
-constexpr uint32_t kKBytes = 3 * kBlock;
-constexpr uint32_t kVBytes = 2 * kBlock;       // value dims 0..63, 64..127
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;
-constexpr uint32_t kOffV = kOffK + kNSK * kKBytes;
-constexpr uint32_t kSmemUsed = kOffV + kNSV * kVBytes;
+constexpr uint32_t kBlock = kBQ * 64 * 2;  // one 128 x 64 bf16 swizzled block: 16 KB
+constexpr uint32_t kQBytes = 3 * kBlock;   // nope lo, nope hi, rope
+constexpr uint32_t kOffQ = 0;              // Q0, then Q1
+constexpr uint32_t kOffRing = 2 * kQBytes;
+constexpr uint32_t kSmemUsed = kOffRing + kRing * kBlock;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256;
+constexpr uint32_t kColS = 0, kColO = 256;  // S_i at kColS + 128 i, O_i at kColO + 128 i
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
@@ -63,34 +74,163 @@ struct AttnArgs {
   int mask_vec;                // rows 16-byte aligned: vector loads
   const uint8_t* tile_class;   // [B, n_qt, n_kv] or null
   __nv_bfloat16* out;          // [B, T, 64*128]
-  int B, T, n_qt, n_kv;
+  int B, T, n_qt, n_kv, n_pairs;
   float scale_log2;            // softmax_scale * log2(e)
   unsigned long long wait_limit_ns;
   unsigned int* err_word;      // device status word
 };
 
-// Tiles of key blocks a query tile visits, in order. Causal: 0..qt. Explicit
-// mask: every key tile whose class is not "all -inf" (all of them when no
-// classification is given).
-struct KvTiles {
-  const uint8_t* cls;  // class row of this (b, qt), or null
-  int end;             // one past the last candidate tile
-  __device__ __forceinline__ int first() const { return next(-1); }
+// Which key tiles the two query tiles of a CTA visit. Causal: tile qt visits
+// 0..qt. Explicit mask: every key tile whose class is not "all -inf" (every
+// tile when no classification is given).
+template <bool kMasked>
+struct PairTiles {
+  int qt[2];
+  bool exists[2];
+  const uint8_t* cls[2];
+  int end;  // one past the last candidate key tile
+
+  __device__ __forceinline__ bool active(int i, int kt) const {
+    if (!exists[i]) return false;
+    if (kMasked) return cls[i] ? cls[i][kt] != kTileSkip : true;
+    return kt <= qt[i];
+  }
   __device__ __forceinline__ int next(int kt) const {
     ++kt;
-    if (cls)
-      while (kt < end && cls[kt] == kTileSkip) ++kt;
+    while (kt < end && !active(0, kt) && !active(1, kt)) ++kt;
     return kt;
   }
-  __device__ __forceinline__ int count() const {
-    int n = 0;
-    for (int kt = first(); kt < end; kt = next(kt)) ++n;
-    return n;
-  }
+  __device__ __forceinline__ int first() const { return next(-1); }
 };
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
   return __uint_as_float(bits16 << 16);
+}
+
+// One row's view of a 128x128 score tile: turns 32 consecutive raw scores
+// (chunk c, already read from tensor memory) into
+// s * scale_log2 + mask * log2(e) - shift, with keys that are excluded
+// (causal, past T, invalid row) at -inf.
+template <bool kMasked>
+struct ScoreChunk {
+  uint8_t cls;                // class of this (query, key) tile
+  bool row_valid;
+  const __nv_bfloat16* mrow;  // mask row at the tile's first key (kMasked)
+  int kvalid;                 // keys of the tile below T
+  int mask_vec;               // 16-byte mask loads allowed
+  int diag_row;               // causal: keys c > diag_row are excluded
+
+  __device__ __forceinline__ void apply(const uint32_t* rr, int c, float scale_log2, float shift,
+                                        float (&x)[32]) const {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = fmaf(__uint_as_float(rr[i]), scale_log2, -shift);
+    if (!kMasked) {
+      if (diag_row < kBKV) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i > diag_row) x[i] = -INFINITY;
+      }
+      return;
+    }
+    if (!row_valid) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] = -INFINITY;
+      return;
+    }
+    if (cls == kTileMixed) {
+      // 8 keys per 16-byte load when rows are 16-byte aligned; a chunk that
+      // starts below T then lies inside the row (mask_ld >= T, mask_ld % 8 ==
+      // 0). Chunks past the last key re-read the last existing one; their keys
+      // are set to -inf below.
+      const int klast = min(kvalid, kBKV) - 1;
+      const int c8_last = klast >> 3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c8 = 4 * c + j;
+        uint32_t ws[4];
+        if (mask_vec) {
+          const uint4 w = ld_nc_v4_ordered(reinterpret_cast<const uint4*>(mrow) + min(c8, c8_last));
+          ws[0] = w.x, ws[1] = w.y, ws[2] = w.z, ws[3] = w.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            ws[e] = ld_nc_u16_ordered(mrow + min(c8 * 8 + 2 * e, klast)) |
+                    (ld_nc_u16_ordered(mrow + min(c8 * 8 + 2 * e + 1, klast)) << 16);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * j + 2 * e] = fmaf(bf16_bits_to_float(ws[e] & 0xffffu), kLog2e, x[8 * j + 2 * e]);
+          x[8 * j + 2 * e + 1] = fmaf(bf16_bits_to_float(ws[e] >> 16), kLog2e, x[8 * j + 2 * e + 1]);
+        }
+      }
+    }
+    if (kvalid < (c + 1) * 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c * 32 + i >= kvalid) x[i] = -INFINITY;
+    }
+  }
+};
+
+// Exponentials moved from the MUFU unit to the FMA pipe (exp2_poly2): pair i
+// of a chunk goes to the polynomial when kUseExp2Poly and (i & kPolyMask) ==
+// kPolyMask. Off: measured on B200 at B=1, T=4096, the softmax warps are bound
+// by issue slots and latency rather than MUFU throughput, and moving one pair
+// in four (or more) to the 10-instruction polynomial made the kernel slower
+// (0.400 ms without, 0.427 ms at 1/4, 0.464 ms at 1/2).
+constexpr bool kUseExp2Poly = false;
+constexpr int kPolyMask = 3;
+
+// Maximum of a row of 128 raw scores; on the diagonal tile keys c > r are
+// excluded (causal).
+template <bool kDiag>
+__device__ __forceinline__ float raw_row_max(const uint32_t (&raw)[kBKV], int r) {
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int i = 0; i < kBKV; i += 8) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v[e] = __uint_as_float(raw[i + e]);
+      if (kDiag && i + e > r) v[e] = -INFINITY;
+    }
+    m4[0] = fmax3(m4[0], v[0], v[1]);
+    m4[1] = fmax3(m4[1], v[2], v[3]);
+    m4[2] = fmax3(m4[2], v[4], v[5]);
+    m4[3] = fmax3(m4[3], v[6], v[7]);
+  }
+  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+
+// Causal tile, 32 raw scores of chunk c: p = 2^(s*scale_log2 - m), packed as
+// bf16 pairs into pk and summed (unrounded, fp32) into the paired partial sums
+// acc. On the diagonal tile keys c > r give 0, and every exponential goes to
+// MUFU (which maps -inf to exactly 0); elsewhere the FMA-pipe polynomial may
+// take some pairs (kUseExp2Poly).
+template <bool kDiag>
+__device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r, float scale_log2,
+                                               float m, uint32_t (&pk)[16], float (&acc)[8]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1;
+    ffma2(x0, x1, __uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1]), scale_log2,
+          scale_log2, -m, -m);
+    float p0, p1;
+    if (kDiag) {
+      if (c * 32 + 2 * i > r) x0 = -INFINITY;
+      if (c * 32 + 2 * i + 1 > r) x1 = -INFINITY;
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    } else if (kUseExp2Poly && (i & kPolyMask) == kPolyMask) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    }
+    const int a = 2 * (i & 3);
+    fadd2(acc[a], acc[a + 1], acc[a], acc[a + 1], p0, p1);
+    pk[i] = pack_bf16x2(p0, p1);
+  }
 }
 
 template <bool kMasked>
@@ -102,10 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full;
-  __shared__ uint64_t k_full[kNSK], k_empty[kNSK];
-  __shared__ uint64_t v_full[kNSV], v_empty[kNSV];
+  __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
   __shared__ uint64_t s_full[2], p_full[2];
-  __shared__ uint64_t o_done;
+  __shared__ uint64_t o_final;
   __shared__ uint64_t drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -115,41 +254,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.x;
-  const int b = blockIdx.y;
-  const int qt = args.n_qt - 1 - int(blockIdx.z);  // longest causal tiles first
-  const int q0 = qt * kBQ;
+
+  // CTA -> (b, h, pair): groups of kHeadGroup heads, longest pairs first
+  // within a group.
+  const int per_group = kHeadGroup * args.n_pairs;
+  const int grp = blockIdx.x / per_group;
+  const int rem = blockIdx.x - grp * per_group;
+  const int b = grp / (kH / kHeadGroup);
+  const int h = (grp % (kH / kHeadGroup)) * kHeadGroup + rem % kHeadGroup;
+  const int pair = args.n_pairs - 1 - rem / kHeadGroup;
   const int bh = b * kH + h;
 
-  KvTiles tiles;
-  if (kMasked) {
-    tiles.cls = args.tile_class ? args.tile_class + (size_t(b) * args.n_qt + qt) * args.n_kv
-                                : nullptr;
-    tiles.end = args.n_kv;
-  } else {
-    tiles.cls = nullptr;
-    tiles.end = qt + 1;
+  PairTiles<kMasked> tiles;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    tiles.qt[i] = 2 * pair + i;
+    tiles.exists[i] = tiles.qt[i] < args.n_qt;
+    tiles.cls[i] = (kMasked && args.tile_class && tiles.exists[i])
+                       ? args.tile_class + (size_t(b) * args.n_qt + tiles.qt[i]) * args.n_kv
+                       : nullptr;
   }
-  const int n = tiles.count();
+  tiles.end = kMasked ? args.n_kv : min(2 * pair + 2, args.n_qt);
+  const bool has_work = tiles.first() < tiles.end;
 
   WaitCtl ctl{&abort_flag, args.wait_limit_ns, kErrKernelAttn, args.err_word};
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(&q_full, 1);
-    for (int s = 0; s < kNSK; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&ring_full[s], 1);
+      mbar_init(&ring_empty[s], 1);
     }
-    for (int s = 0; s < kNSV; ++s) {
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
-    }
-    mbar_init(&o_done, 1);
+    mbar_init(&o_final, 1);
     mbar_init(&drain_bar, 1);
     fence_barrier_init();
   }
@@ -162,106 +303,173 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
+  if (warp < 4) {
+  // Warpgroup 0 (TMA producer, MMA issuer, two idle warps) hands registers
+  // to the two softmax warpgroups.
+  setmaxnreg_dec<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n > 0) {
+    if (lane == 0 && has_work) {
       prefetch_tensormap(&tmQn);
       prefetch_tensormap(&tmQp);
       prefetch_tensormap(&tmKn);
       prefetch_tensormap(&tmKp);
       prefetch_tensormap(&tmV);
-      uint8_t* sQ = smem + kOffQ;
-      mbar_arrive_expect_tx(&q_full, kQBytes);
-      tma_load_3d(sQ, &tmQn, &q_full, 0, q0, bh);
-      tma_load_3d(sQ + kBlock, &tmQn, &q_full, 64, q0, bh);
-      tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full, 0, q0, bh);
-      uint32_t k_issued = 0, k_par = 0, v_issued = 0, v_par = 0;
+      const uint32_t nq = tiles.exists[1] ? 2u : 1u;
+      mbar_arrive_expect_tx(&q_full, nq * kQBytes);
+      for (uint32_t i = 0; i < nq; ++i) {
+        uint8_t* sQ = smem + kOffQ + i * kQBytes;
+        const int q0 = tiles.qt[i] * kBQ;
+        tma_load_3d(sQ, &tmQn, &q_full, 0, q0, bh);
+        tma_load_3d(sQ + kBlock, &tmQn, &q_full, 64, q0, bh);
+        tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full, 0, q0, bh);
+      }
+      uint32_t issued = 0, issued_par = 0;
+      uint32_t s = 0;  // block sequence number
       bool ok = true;
-      int j = 0;
-      for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt), ++j) {
+      for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt)) {
         const int k0 = kt * kBKV;
-        const int sk = j % kNSK;
-        const uint32_t pk = (j / kNSK) & 1;
-        if (!mbar_wait(&k_empty[sk], pk ^ 1u, ctl, 1)) { ok = false; break; }
-        uint8_t* sK = smem + kOffK + sk * kKBytes;
-        mbar_arrive_expect_tx(&k_full[sk], kKBytes);
-        tma_load_3d(sK, &tmKn, &k_full[sk], 0, k0, bh);
-        tma_load_3d(sK + kBlock, &tmKn, &k_full[sk], 64, k0, bh);
-        tma_load_3d(sK + 2 * kBlock, &tmKp, &k_full[sk], 0, k0, b);
-        k_issued |= 1u << sk;
-        k_par = (k_par & ~(1u << sk)) | (pk << sk);
-
-        const int sv = j % kNSV;
-        const uint32_t pv = (j / kNSV) & 1;
-        if (!mbar_wait(&v_empty[sv], pv ^ 1u, ctl, 2)) { ok = false; break; }
-        uint8_t* sV = smem + kOffV + sv * kVBytes;
-        mbar_arrive_expect_tx(&v_full[sv], kVBytes);
-        tma_load_3d(sV, &tmV, &v_full[sv], 0, k0, bh);
-        tma_load_3d(sV + kBlock, &tmV, &v_full[sv], 64, k0, bh);
-        v_issued |= 1u << sv;
-        v_par = (v_par & ~(1u << sv)) | (pv << sv);
+#pragma unroll 1
+        for (int i = 0; i < kBlocksPerTile; ++i, ++s) {
+          const uint32_t slot = s % kRing;
+          const uint32_t par = (s / kRing) & 1u;
+          if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
+          uint8_t* dst = smem + kOffRing + slot * kBlock;
+          mbar_arrive_expect_tx(&ring_full[slot], kBlock);
+          switch (i) {
+            case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0, bh); break;
+            case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0, bh); break;
+            case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0, b); break;
+            default: {
+              // V for 64 keys, all 128 value dims: two 64 x 64 boxes, 8 KB apart
+              const int kv = k0 + (i - 3) * 64;
+              tma_load_3d(dst, &tmV, &ring_full[slot], 0, kv, bh);
+              tma_load_3d(dst + kBlock / 2, &tmV, &ring_full[slot], 64, kv, bh);
+              break;
+            }
+          }
+          issued |= 1u << slot;
+          issued_par = (issued_par & ~(1u << slot)) | (par << slot);
+        }
       }
       if (!ok) {
+        // let the copies already issued land before the CTA's memory goes away
         int zero = 0;
         WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
-        mbar_wait(&q_full, 0, drain, 3);
-        for (int s = 0; s < kNSK; ++s)
-          if (k_issued & (1u << s)) mbar_wait(&k_full[s], (k_par >> s) & 1u, drain, 4);
-        for (int s = 0; s < kNSV; ++s)
-          if (v_issued & (1u << s)) mbar_wait(&v_full[s], (v_par >> s) & 1u, drain, 5);
+        mbar_wait(&q_full, 0, drain, 2);
+        for (int k = 0; k < kRing; ++k)
+          if (issued & (1u << k)) mbar_wait(&ring_full[k], (issued_par >> k) & 1u, drain, 3);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
+    if (lane == 0 && has_work) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBQ, kBKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, kDV, false, true);
-      const uint32_t sQ = smem_u32(smem + kOffQ);
+      const uint32_t ring0 = smem_u32(smem + kOffRing);
       bool ok = mbar_wait(&q_full, 0, ctl, 10);
       bool issued_any = false;
+      uint32_t n_pv[2] = {0, 0};  // PVs issued per query tile
+      int prev = -1;               // previous visited key tile
+      bool prev_act[2] = {false, false};
+      uint32_t prev_base = 0;      // block sequence number of prev's first block
+      bool prev_v_ready = false;
 
-      auto issue_pv = [&](int i) -> bool {
-        const int sv = i % kNSV;
-        const int pb = i & 1;
-        if (!mbar_wait(&p_full[pb], (i >> 1) & 1, ctl, 11)) return false;
-        if (!mbar_wait(&v_full[sv], (i / kNSV) & 1, ctl, 12)) return false;
-        tc_fence_after();
-        const uint32_t sV = smem_u32(smem + kOffV + sv * kVBytes);
-        const uint32_t p_tmem = tmem_base + kColS0 + pb * 128;
-#pragma unroll
-        for (int kk = 0; kk < kBKV / 16; ++kk) {
-          // 16 keys = 8 packed TMEM columns of P; 16 V rows of 128 bytes.
-          const uint64_t vd = sdesc_sw128(sV + kk * 16 * 128, kBlock, 1024);
-          mma_ts(tmem_base + kColO, p_tmem + kk * 8, vd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&o_done);
-        mma_commit(&v_empty[sv]);
-        return true;
+      auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
+        return mbar_wait(&ring_full[seq % kRing], (seq / kRing) & 1u, ctl, site);
       };
+      auto block_addr = [&](uint32_t seq) -> uint32_t { return ring0 + (seq % kRing) * kBlock; };
 
-      int j = 0;
-      for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt), ++j) {
-        const int sk = j % kNSK;
-        const int sb = j & 1;
-        if (!mbar_wait(&k_full[sk], (j / kNSK) & 1, ctl, 13)) { ok = false; break; }
+      // O_i += P_i V for the key tile whose blocks start at `base`.
+      auto issue_pv = [&](int i, uint32_t base) -> bool {
+        if (!mbar_wait(&p_full[i], n_pv[i] & 1u, ctl, 11)) return false;
+        if (!prev_v_ready) {
+          if (!wait_block(base + 3, 12) || !wait_block(base + 4, 12)) return false;
+          prev_v_ready = true;
+        }
         tc_fence_after();
-        const uint32_t sK = smem_u32(smem + kOffK + sk * kKBytes);
-        const uint32_t s_tmem = tmem_base + kColS0 + sb * 128;
+        const uint32_t p_tmem = tmem_base + kColS + 128 * i;
+        const uint32_t o_tmem = tmem_base + kColO + 128 * i;
+        // Each V block holds 64 keys x 128 value dims, MN-major: value dims
+        // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB apart
+        // (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
 #pragma unroll
-        for (int blk = 0; blk < 3; ++blk) {
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t vb = block_addr(base + 3 + half);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
-            const uint64_t kd = sdesc_sw128(sK + blk * kBlock + kk * 32, 16, 1024);
-            mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
+            const uint32_t acc = (n_pv[i] > 0 || half > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
+            mma_ts(o_tmem, p_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
           }
         }
-        issued_any = true;
-        mma_commit(&s_full[sb]);
-        mma_commit(&k_empty[sk]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        ++n_pv[i];
+        return true;
+      };
+      auto release_v = [&](uint32_t base) {
+        mma_commit(&ring_empty[(base + 3) % kRing]);
+        mma_commit(&ring_empty[(base + 4) % kRing]);
+      };
+
+      uint32_t base = 0;
+      for (int kt = tiles.first(); ok && kt < tiles.end;
+           kt = tiles.next(kt), base += kBlocksPerTile) {
+        const bool act[2] = {tiles.active(0, kt), tiles.active(1, kt)};
+        const uint32_t k_addr[3] = {block_addr(base), block_addr(base + 1),
+                                    block_addr(base + 2)};
+        bool k_ready = false;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (prev >= 0 && prev_act[i]) {
+            if (!issue_pv(i, prev_base)) { ok = false; break; }
+            issued_any = true;
+          }
+          if (act[i]) {
+            // K is waited for only now, after the previous tile's first PV:
+            // its slots free up late in the previous iteration.
+            if (!k_ready) {
+              if (!wait_block(base, 13) || !wait_block(base + 1, 13) ||
+                  !wait_block(base + 2, 13)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              k_ready = true;
+            }
+            const uint32_t sQ = smem_u32(smem + kOffQ + i * kQBytes);
+            const uint32_t s_tmem = tmem_base + kColS + 128 * i;
+#pragma unroll
+            for (int blk = 0; blk < 3; ++blk) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
+                const uint64_t kd = sdesc_sw128(k_addr[blk] + kk * 32, 16, 1024);
+                mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
+              }
+            }
+            issued_any = true;
+            mma_commit(&s_full[i]);
+          }
+        }
+        if (!ok) break;
+        if (prev >= 0) release_v(prev_base);
+        mma_commit(&ring_empty[base % kRing]);
+        mma_commit(&ring_empty[(base + 1) % kRing]);
+        mma_commit(&ring_empty[(base + 2) % kRing]);
+        prev = kt;
+        prev_act[0] = act[0];
+        prev_act[1] = act[1];
+        prev_base = base;
+        prev_v_ready = false;
       }
-      if (ok && !issue_pv(n - 1)) ok = false;
+      if (ok && prev >= 0) {
+        for (int i = 0; i < 2 && ok; ++i)
+          if (prev_act[i]) ok = issue_pv(i, prev_base);
+        if (ok) {
+          release_v(prev_base);
+          mma_commit(&o_final);
+        }
+      }
       if (!ok && issued_any) {
         mma_commit(&drain_bar);
         int zero = 0;
@@ -269,91 +477,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&drain_bar, 0, drain, 14);
       }
     }
+  }
+  named_barrier_sync(kBarTeardown, kThreads);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
   } else {
+  setmaxnreg_inc<kRegsSoftmax>();
+  {
     // ------------------------------------------------------------ softmax / epilogue
-    const int quad = warp & 3;
+    const int wi = (warp - 4) >> 2;  // query tile of this warpgroup
+    const int quad = warp & 3;       // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;  // row within the tile == TMEM lane
-    const int q = q0 + r;
+    const int qt = tiles.qt[wi];
+    const int q = qt * kBQ + r;
     const uint32_t lane_base = tmem_addr(tmem_base, quad * 32, 0);
-    const bool row_valid = q < args.T;
+    const uint32_t colS = kColS + 128 * wi;
+    const uint32_t colO = kColO + 128 * wi;
+    const bool row_valid = tiles.exists[wi] && q < args.T;
     const __nv_bfloat16* mrow =
         (kMasked && row_valid) ? args.mask + (size_t(b) * args.T + q) * args.mask_ld : nullptr;
 
     float m = -INFINITY;  // running max, log2 units
     float l = 0.f;        // running sum of p (fp32, unrounded)
     bool ok = true;
-    int j = 0;
-    for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt), ++j) {
-      const int sb = j & 1;
+    uint32_t n = 0;
+    for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) {
+      if (!tiles.active(wi, kt)) continue;
       const int k0 = kt * kBKV;
-      if (!mbar_wait_warp(&s_full[sb], (j >> 1) & 1, ctl, 20)) { ok = false; break; }
+      if (!mbar_wait_warp(&s_full[wi], n & 1u, ctl, 20)) { ok = false; break; }
       tc_fence_after();
-      // scores in log2 units, with the explicit mask added chunk by chunk
-      const uint8_t cls =
-          (kMasked && row_valid) ? (tiles.cls ? tiles.cls[kt] : uint8_t(kTileMixed))
-                                   : uint8_t(kTileZero);
-      const int kvalid = args.T - k0;  // keys of this tile that exist
-      // 8 keys per 16-byte load when the rows are 16-byte aligned; a chunk
-      // that starts below T then lies inside the row (mask_ld >= T and
-      // mask_ld % 8 == 0).
-      const uint4* mv = reinterpret_cast<const uint4*>(mrow + k0);
-      const int c8_last = (min(kvalid, kBKV) - 1) >> 3;
-      float x[kBKV];
+      // The 128 scores of this thread's row are read from tensor memory once
+      // and kept in registers for both passes (row maximum, exponentials).
+      ScoreChunk<kMasked> sc;
+      sc.cls = (kMasked && row_valid)
+                   ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed))
+                   : uint8_t(kTileZero);
+      sc.row_valid = row_valid;
+      sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
+      sc.kvalid = args.T - k0;
+      sc.mask_vec = args.mask_vec;
+      sc.diag_row = (!kMasked && kt == qt) ? r : kBKV;  // causal: key c allowed iff c <= r
+      const bool causal_fast = !kMasked && args.scale_log2 > 0.f;
+      const bool diag = !kMasked && kt == qt;
+      uint32_t raw[kBKV];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(lane_base + kColS0 + sb * 128 + c * 32, rr);
-        tmem_ld_wait();
-        reg_fence(rr);
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
+      tmem_ld_wait();
+      reg_fence(raw);
+      float mt;
+      if (causal_fast) {
+        // positive scale: the maximum of the raw scores gives the maximum of
+        // the scaled ones
+        mt = diag ? raw_row_max<true>(raw, r) : raw_row_max<false>(raw, r);
+        mt *= args.scale_log2;
+      } else {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rr[i]) * args.scale_log2;
-        if (cls == kTileMixed) {
+        for (int c = 0; c < 4; ++c) {
+          float x[32];
+          sc.apply(raw + c * 32, c, args.scale_log2, 0.f, x);
 #pragma unroll
-          for (int c8 = 4 * c; c8 < 4 * c + 4; ++c8) {
-            // Chunks past the last key re-read the last existing chunk; their
-            // keys are set to -inf below.
-            const int c8c = min(c8, c8_last);
-            uint32_t ws[4];
-            if (args.mask_vec) {
-              const uint4 w = ld_nc_v4_ordered(mv + c8c);
-              ws[0] = w.x, ws[1] = w.y, ws[2] = w.z, ws[3] = w.w;
-            } else {
-              // rows not 16-byte aligned: element loads, clamped to the row
-              const __nv_bfloat16* mc = mrow + k0;
-              const int klast = min(kvalid, kBKV) - 1;
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                ws[e] = ld_nc_u16_ordered(mc + min(c8 * 8 + 2 * e, klast)) |
-                        (ld_nc_u16_ordered(mc + min(c8 * 8 + 2 * e + 1, klast)) << 16);
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              x[c8 * 8 + 2 * e] += bf16_bits_to_float(ws[e] & 0xffffu) * kLog2e;
-              x[c8 * 8 + 2 * e + 1] += bf16_bits_to_float(ws[e] >> 16) * kLog2e;
-            }
+          for (int i = 0; i < 32; i += 8) {
+            m4[0] = fmax3(m4[0], x[i], x[i + 1]);
+            m4[1] = fmax3(m4[1], x[i + 2], x[i + 3]);
+            m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
+            m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
           }
         }
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      if (!kMasked) {
-        if (kt == qt) {  // diagonal tile: key k0+c allowed iff c <= r
-#pragma unroll
-          for (int c = 0; c < kBKV; ++c)
-            if (c > r) x[c] = -INFINITY;
-        }
-      } else if (!row_valid) {
-#pragma unroll
-        for (int c = 0; c < kBKV; ++c) x[c] = -INFINITY;
-      } else if (kvalid < kBKV) {
-#pragma unroll
-        for (int c = 0; c < kBKV; ++c)
-          if (c >= kvalid) x[c] = -INFINITY;
-      }
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBKV; ++c) mt = fmaxf(mt, x[c]);
       float alpha = 1.f;
       float m_new = m;
-      if (j == 0) {
+      if (n == 0) {
         m_new = mt;
       } else if (mt > m + kRescaleThreshold) {
         m_new = mt;
@@ -362,46 +560,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       m = m_new;
 
-      if (j >= 1) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled.
-        if (!mbar_wait_warp(&o_done, (j - 1) & 1, ctl, 21)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(lane_base + kColO + c * 32, rr);
-            tmem_ld_wait();
-            reg_fence(rr);
+      // P as bf16 pairs over the first 64 columns of the S buffer (every score
+      // is in registers by now), 32 keys per store.
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(lane_base + kColO + c * 32, rr);
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t* rc = raw + c * 32;
+        uint32_t pk[16];
+        if (causal_fast) {
+          if (diag)
+            p_chunk_causal<true>(rc, c, r, args.scale_log2, m_use, pk, acc);
+          else
+            p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
+        } else {
+          float x[32];
+          sc.apply(rc, c, args.scale_log2, m_use, x);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(x[2 * i]);
+            const float p1 = fast_exp2(x[2 * i + 1]);
+            fadd2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)],
+                  acc[2 * (i & 3) + 1], p0, p1);
+            pk[i] = pack_bf16x2(p0, p1);
           }
         }
+        tmem_st16(lane_base + colS + 16 * c, pk);
       }
-      // P_j as bf16 pairs over the first 64 columns of its S buffer, written
-      // 32 columns (64 keys) at a time.
-      float rowsum = 0.f;
+      const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                           ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+
+      // O holds P_{n-1} V_{n-1} here: that PV was issued before this S, and
+      // the commit behind s_full covers every earlier MMA. The rescale lands
+      // before PV_n, which waits for p_full below.
+      if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(lane_base + colO + c * 32, rr);
+          tmem_ld_wait();
+          reg_fence(rr);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = fast_exp2(x[64 * half + 2 * c] - m_use);
-          const float p1 = fast_exp2(x[64 * half + 2 * c + 1] - m_use);
-          rowsum += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32(lane_base + colO + c * 32, rr);
         }
-        tmem_st32(lane_base + kColS0 + sb * 128 + 32 * half, pk);
       }
       l = l * alpha + rowsum;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[wi]);
+      ++n;
     }
 
     // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]
-    const bool have = ok && n > 0 && mbar_wait_warp(&o_done, (n - 1) & 1, ctl, 22);
+    const bool have = ok && n > 0 && mbar_wait_warp(&o_final, 0, ctl, 22);
     if (have) tc_fence_after();
     if (n == 0 || have) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
@@ -410,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
         if (n > 0) {
-          tmem_ld32(lane_base + kColO + c * 32, rr);
+          tmem_ld32(lane_base + colO + c * 32, rr);
           tmem_ld_wait();
           reg_fence(rr);
         } else {
@@ -434,10 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+  named_barrier_sync(kBarTeardown, kThreads);
   }
 }
 
@@ -453,7 +661,8 @@ __global__ void __launch_bounds__(256)
   const int q0 = qt * kBQ, k0 = kt * kBKV;
   const int rows = min(kBQ, T - q0);
   const int cols = min(kBKV, T - k0);
-  const uint16_t* base = reinterpret_cast<const uint16_t*>(mask) + (size_t(b) * T + q0) * mask_ld + k0;
+  const uint16_t* base =
+      reinterpret_cast<const uint16_t*>(mask) + (size_t(b) * T + q0) * mask_ld + k0;
   bool all_ninf = true, all_zero = true;
   if (vec && cols == kBKV) {
     // 16 uint4 per row
@@ -491,10 +700,12 @@ bool mask_rows_vec_ok(const void* mask, int64_t mask_ld) {
   return (reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (mask_ld % 8) == 0;
 }
 
-bool make_map_3d(CUtensorMap* m, const void* p, int inner, int T, int outer) {
+// [outer][T][inner] bf16 tensor, boxes of 64 (inner) x box_rows (T) x 1.
+bool make_map_3d(CUtensorMap* m, const void* p, int inner, int T, int outer,
+                 uint32_t box_rows = kBQ) {
   const uint64_t dims[3] = {uint64_t(inner), uint64_t(T), uint64_t(outer)};
   const uint64_t strides[2] = {uint64_t(inner) * 2, uint64_t(inner) * 2 * uint64_t(T)};
-  const uint32_t box[3] = {64, kBQ, 1};
+  const uint32_t box[3] = {64, box_rows, 1};
   return encode_tmap_bf16(m, p, 3, dims, strides, box, true);
 }
 
@@ -525,7 +736,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   const int BH = B * kH;
   if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
       !make_map_3d(&tmKn, k_nope, kDN, T, BH) || !make_map_3d(&tmKp, k_pe, kDR, T, B) ||
-      !make_map_3d(&tmV, v, kDV, T, BH))
+      !make_map_3d(&tmV, v, kDV, T, BH, 64))
     return cudaErrorInvalidValue;
   auto kern = mask ? mla_attn_prefill_kernel<true> : mla_attn_prefill_kernel<false>;
   static unsigned attr_done[2] = {0, 0};
@@ -542,11 +753,13 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   a.T = T;
   a.n_qt = (T + kBQ - 1) / kBQ;
   a.n_kv = a.n_qt;
+  a.n_pairs = (a.n_qt + 1) / 2;
   a.scale_log2 = softmax_scale * kLog2e;
   a.wait_limit_ns = wait_limit_ns;
   a.err_word = err_word;
-  dim3 grid(kH, B, a.n_qt);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, a);
+  const long long ctas = (long long)B * kH * a.n_pairs;
+  if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
+  kern<<<unsigned(ctas), kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, a);
   return cudaGetLastError();
 }
 
