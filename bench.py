@@ -69,6 +69,25 @@ def row_flops(i, T):
     return H * (i + 1) * 2 * (DQK + DV) + 2 * K_OPROJ * D_MODEL
 
 
+# ---------------------------------------------------------------- multi-rank
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (identity for one rank). The timed
+    region of a multi-GPU run is the slowest rank's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step: float, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own batch;
+    the job takes the slowest rank's time."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- helpers
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -305,17 +324,13 @@ def run_ours(args, w, rank, world, local_rank):
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     oproj_ms = [e[1].elapsed_time(e[2]) for e in evs]
     step_ms = [a + b for a, b in zip(attn_ms, oproj_ms)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
     vl = d["valid_len"].tolist() if d["valid_len"] is not None else None
     fa = attn_flops(B, T, vl)
     fo = oproj_flops(B * T)
     flops_step = fa + fo
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, flops_step, args.steps, total_ms)
 
     # e2e through mla_attn_oproj from pinned host buffers (W_o stays resident)
     e2e = None
@@ -347,12 +362,8 @@ def run_ours(args, w, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * flops_step * n_e2e / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_tflops(world, flops_step, n_e2e, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e2e_ms / n_e2e, "call": "mla_attn_oproj",
                "note": "per step: pinned H2D of the activations (and mask), the fused call, "
