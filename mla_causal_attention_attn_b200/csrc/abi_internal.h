@@ -1,0 +1,47 @@
+// abi_internal.h -- host-side helpers shared by the C entry points
+// (argument checks, device checks, the device status word, the attention
+// launch sequence). Defined in mla_abi.cu.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+namespace abi {
+
+constexpr int kMaxB = 65535;
+constexpr int kMaxT = 65535 * 128;
+constexpr int64_t kMaxM = (int64_t(1) << 31) - 129;
+
+// Device address of the library's status word on the current device (fetched
+// once per device), or null.
+unsigned int* device_error_word();
+
+// Per-wait limit of the kernels' bounded waits (MLA_WAIT_LIMIT_NS, else 1 s).
+unsigned long long wait_limit_ns();
+
+bool aligned16(const void* p);
+size_t round_up(size_t x, size_t a);
+
+// MLA_ERR_UNSUPPORTED_DEVICE unless the current device is CC 10.0.
+mla_status_t check_device();
+
+// Pointer, shape, scale and alignment checks shared by the attention calls.
+mla_status_t check_attn_args(const void* q_nope, const void* q_pe, const void* k_nope,
+                             const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
+                             int B, int T, float softmax_scale, const void* out);
+
+mla_status_t from_cuda(cudaError_t e);
+
+// Mask-tile classification (when mask is given, into `cls`) followed by the
+// attention kernel writing the merged heads to `out`.
+mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
+                           const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
+                           int B, int T, float softmax_scale, void* cls, void* out,
+                           cudaStream_t stream);
+
+}  // namespace abi
+}  // namespace mla

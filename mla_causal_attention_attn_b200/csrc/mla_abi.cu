@@ -5,6 +5,7 @@
 #include <cstdlib>
 
 #include "../../include/mla.h"
+#include "abi_internal.h"
 #include "attn_prefill.h"
 #include "host_util.h"
 #include "oproj_gemm.h"
@@ -15,7 +16,7 @@ namespace mla {
 // The library's device status word (one per device that loads the library).
 __device__ unsigned int g_device_error = 0;
 
-namespace {
+namespace abi {
 
 // Device address of g_device_error for the current device, fetched once per
 // device; null if the runtime cannot provide it.
@@ -33,10 +34,6 @@ unsigned int* device_error_word() {
   }
   return p;
 }
-
-constexpr int kMaxB = 65535;
-constexpr int kMaxT = 65535 * 128;
-constexpr int64_t kMaxM = (int64_t(1) << 31) - 129;
 
 unsigned long long wait_limit_ns() {
   // MLA_WAIT_LIMIT_NS overrides the per-wait limit (read once).
@@ -93,10 +90,11 @@ mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_n
                                        wait_limit_ns(), device_error_word(), stream));
 }
 
-}  // namespace
+}  // namespace abi
 }  // namespace mla
 
 using namespace mla;
+using namespace mla::abi;
 
 extern "C" {
 
