@@ -142,6 +142,38 @@ mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
                             int T, float softmax_scale, const mla_bf16* W_o, void* workspace,
                             size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
 
+/* Largest B*T mla_attn_oproj_noalloc accepts (its fixed scratch holds the
+ * merged attention output of this many tokens: 64 MiB). */
+#define MLA_NOALLOC_MAX_TOKENS 4096
+
+/*
+ * mla_attn_oproj without a workspace argument, for callers that cannot
+ * allocate device memory at all (for example code running inside a host
+ * framework that owns every device allocation, or a plugin that is handed its
+ * inputs and outputs and nothing else). The pages have no counterpart of
+ * this call; it exists only because of how such callers are built.
+ *
+ * Arguments, layouts and results are those of mla_attn_oproj minus
+ * `workspace`/`workspace_bytes`. The scratch is one fixed device array inside
+ * the library (64 MiB + 64 KiB) that every GPU which loads the library holds
+ * until the process exits; this call allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library routine).
+ *  - B*T above MLA_NOALLOC_MAX_TOKENS -> MLA_ERR_WORKSPACE (the fixed scratch
+ *    is too small); every other error as in mla_attn_oproj.
+ *  - The first call on a device looks up the scratch's device address on that
+ *    device (cudaGetSymbolAddress, which may load the library's module there):
+ *    make that first call before any stream capture.
+ *  - All calls share the one scratch array, which keeps the previous call's
+ *    contents (nothing in it needs to start at zero). Calls whose GPU work can
+ *    overlap -- different streams, or different host threads, on one device --
+ *    race on it and must be serialised by the caller.
+ */
+mla_status_t mla_attn_oproj_noalloc(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                    const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                    const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld,
+                                    int B, int T, float softmax_scale, const mla_bf16* W_o,
+                                    mla_bf16* out, mla_stream_t stream);
+
 /*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns MLA_ERR_TIMEOUT if any kernel of this library gave

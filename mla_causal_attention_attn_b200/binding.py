@@ -46,6 +46,9 @@ _SIGNATURES = {
     "mla_attn_oproj": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_float, _VP, _VP, ctypes.c_size_t, _VP,
                                       _VP]),
+    "mla_attn_oproj_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_float, _VP,
+                                              _VP, _VP]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_abi_version": (ctypes.c_int, []),
@@ -193,6 +196,34 @@ def attn_oproj(q_nope, q_pe, k_nope, k_pe, v, W_o, mask=None, softmax_scale=None
                             _ptr(mask), mask_ld, B, T, scale, _ptr(W_o), _ptr(workspace),
                             ws_bytes, _ptr(out), _stream_handle(stream))
     _check("mla_attn_oproj", st)
+    return out
+
+
+NOALLOC_MAX_TOKENS = 4096  # MLA_NOALLOC_MAX_TOKENS
+
+
+def attn_oproj_noalloc(q_nope, q_pe, k_nope, k_pe, v, W_o, mask=None, softmax_scale=None,
+                       out=None, stream=None):
+    """Whole path through ``mla_attn_oproj_noalloc``: no workspace; the library
+    uses its own fixed scratch (B*T <= 4096 tokens). Meant for callers that
+    cannot allocate device memory; ``out`` should then be passed in."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    st = lib.mla_attn_oproj_noalloc(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                    _ptr(mask), mask_ld, B, T, scale, _ptr(W_o), _ptr(out),
+                                    _stream_handle(stream))
+    _check("mla_attn_oproj_noalloc", st)
     return out
 
 
