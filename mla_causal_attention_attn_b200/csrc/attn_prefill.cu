@@ -206,10 +206,12 @@ __device__ __forceinline__ float raw_row_max(const uint32_t (&raw)[kBKV], int r)
 // bf16 pairs into pk and summed (unrounded, fp32) into the paired partial sums
 // acc. On the diagonal tile keys c > r give 0, and every exponential goes to
 // MUFU (which maps -inf to exactly 0); elsewhere the FMA-pipe polynomial may
-// take some pairs (kUseExp2Poly).
-template <bool kDiag>
+// take some pairs (kUseExp2Poly). With kTrackMax, xmax[0..1] also collect the
+// largest s*scale_log2 - m seen (the caller's running-max check).
+template <bool kDiag, bool kTrackMax = false>
 __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r, float scale_log2,
-                                               float m, uint32_t (&pk)[16], float (&acc)[8]) {
+                                               float m, uint32_t (&pk)[16], float (&acc)[8],
+                                               float* xmax = nullptr) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     float x0, x1;
@@ -219,6 +221,9 @@ __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r
     if (kDiag) {
       if (c * 32 + 2 * i > r) x0 = -INFINITY;
       if (c * 32 + 2 * i + 1 > r) x1 = -INFINITY;
+    }
+    if (kTrackMax) xmax[i & 1] = fmax3(xmax[i & 1], x0, x1);
+    if (kDiag) {
       p0 = fast_exp2(x0);
       p1 = fast_exp2(x1);
     } else if (kUseExp2Poly && (i & kPolyMask) == kPolyMask) {
@@ -527,6 +532,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
       tmem_ld_wait();
       reg_fence(raw);
+      float alpha = 1.f;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
+      // Causal tiles after the first: one pass against the running max m,
+      // writing P while tracking the tile's largest s*scale - m. Only if that
+      // exceeds the 2^8 headroom is the tile redone exactly below (new max,
+      // O rescaled). The first tile and the masked kernel always take the
+      // exact two-pass route.
+      bool exact = !(causal_fast && n > 0 && m > -INFINITY);
+      if (!exact) {
+        float xmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+          if (diag)
+            p_chunk_causal<true, true>(raw + c * 32, c, r, args.scale_log2, m, pk, acc, xmax);
+          else
+            p_chunk_causal<false, true>(raw + c * 32, c, r, args.scale_log2, m, pk, acc, xmax);
+          tmem_st16(lane_base + colS + 16 * c, pk);
+        }
+        exact = __any_sync(0xffffffffu, fmaxf(xmax[0], xmax[1]) > kRescaleThreshold);
+        if (exact) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        }
+      }
+      if (exact) {
       float mt;
       if (causal_fast) {
         // positive scale: the maximum of the raw scores gives the maximum of
@@ -549,7 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      float alpha = 1.f;
       float m_new = m;
       if (n == 0) {
         m_new = mt;
@@ -562,7 +592,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // P as bf16 pairs over the first 64 columns of the S buffer (every score
       // is in registers by now), 32 keys per store.
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const uint32_t* rc = raw + c * 32;
@@ -586,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(lane_base + colS + 16 * c, pk);
       }
+      }  // exact
       const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
                            ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 
