@@ -249,8 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t q_full;
   __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
   __shared__ uint64_t s_full[2], p_full[2];
-  __shared__ uint64_t o_final;
-  __shared__ uint64_t drain_bar;
+  __shared__ uint64_t o_final[2];
+  __shared__ uint64_t drain_bar[2];
+  __shared__ uint64_t s_issued[2];  // issuer i has issued (or skipped) S of its next tile
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -289,14 +290,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&q_full, 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&ring_full[s], 1);
-      mbar_init(&ring_empty[s], 1);
+      // released once by each query tile's MMA issuer
+      mbar_init(&ring_empty[s], tiles.exists[1] ? 2 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
     }
-    mbar_init(&o_final, 1);
-    mbar_init(&drain_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_final[i], 1);
+      mbar_init(&drain_bar[i], 1);
+      mbar_init(&s_issued[i], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -332,8 +337,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0, issued_par = 0;
       uint32_t s = 0;  // block sequence number
       bool ok = true;
+      // Key tiles are prefetched into L2 two visited tiles ahead of their
+      // loads (the first CTA of a head group to reach a tile otherwise waits
+      // on DRAM with the ring slots already committed).
+      auto prefetch_tile = [&](int pt) {
+        if (pt >= tiles.end) return;
+        const int p0 = pt * kBKV;
+        tma_prefetch_l2_3d(&tmKn, 0, p0, bh);
+        tma_prefetch_l2_3d(&tmKn, 64, p0, bh);
+        tma_prefetch_l2_3d(&tmKp, 0, p0, b);
+        tma_prefetch_l2_3d(&tmV, 0, p0, bh);
+        tma_prefetch_l2_3d(&tmV, 64, p0, bh);
+        tma_prefetch_l2_3d(&tmV, 0, p0 + 64, bh);
+        tma_prefetch_l2_3d(&tmV, 64, p0 + 64, bh);
+      };
+      int pf = tiles.next(tiles.first());
+      prefetch_tile(pf);
       for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt)) {
         const int k0 = kt * kBKV;
+        if (pf < tiles.end) {
+          pf = tiles.next(pf);
+          prefetch_tile(pf);
+        }
 #pragma unroll 1
         for (int i = 0; i < kBlocksPerTile; ++i, ++s) {
           const uint32_t slot = s % kRing;
@@ -366,120 +391,121 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (issued & (1u << k)) mbar_wait(&ring_full[k], (issued_par >> k) & 1u, drain, 3);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && has_work) {
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues the MMAs of query tile 0, warp 2 those of query tile 1,
+    // so a tile's PV is never held up behind the other tile's queued MMAs in
+    // one issuing thread. Per visited key tile j an issuer runs
+    //   O += P_{j-1} V_{j-1}, release V_{j-1};  S = Q K_j^T, release K_j.
+    // The S MMAs keep a strict order S0_0, S1_0, S0_1, S1_1, ... (s_issued),
+    // which keeps the two softmax warpgroups out of phase.
+    const int qi = warp - 1;
+    if (lane == 0 && has_work && tiles.exists[qi]) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBQ, kBKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, kDV, false, true);
       const uint32_t ring0 = smem_u32(smem + kOffRing);
+      const uint32_t sQ = smem_u32(smem + kOffQ + qi * kQBytes);
+      const uint32_t s_tmem = tmem_base + kColS + 128 * qi;  // S, and P over it
+      const uint32_t o_tmem = tmem_base + kColO + 128 * qi;
+      const bool pair = tiles.exists[1];
       bool ok = mbar_wait(&q_full, 0, ctl, 10);
       bool issued_any = false;
-      uint32_t n_pv[2] = {0, 0};  // PVs issued per query tile
-      int prev = -1;               // previous visited key tile
-      bool prev_act[2] = {false, false};
-      uint32_t prev_base = 0;      // block sequence number of prev's first block
-      bool prev_v_ready = false;
+      uint32_t n_pv = 0;       // PVs issued
+      uint32_t n_tiles = 0;    // visited key tiles so far
+      int prev = -1;           // previous visited key tile
+      bool prev_act = false;   // did this query tile use it
+      uint32_t prev_base = 0;  // block sequence number of prev's first block
 
       auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
         return mbar_wait(&ring_full[seq % kRing], (seq / kRing) & 1u, ctl, site);
       };
       auto block_addr = [&](uint32_t seq) -> uint32_t { return ring0 + (seq % kRing) * kBlock; };
-
-      // O_i += P_i V for the key tile whose blocks start at `base`.
-      auto issue_pv = [&](int i, uint32_t base) -> bool {
-        if (!mbar_wait(&p_full[i], n_pv[i] & 1u, ctl, 11)) return false;
-        if (!prev_v_ready) {
-          if (!wait_block(base + 3, 12) || !wait_block(base + 4, 12)) return false;
-          prev_v_ready = true;
-        }
-        tc_fence_after();
-        const uint32_t p_tmem = tmem_base + kColS + 128 * i;
-        const uint32_t o_tmem = tmem_base + kColO + 128 * i;
-        // Each V block holds 64 keys x 128 value dims, MN-major: value dims
-        // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB apart
-        // (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t vb = block_addr(base + 3 + half);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (n_pv[i] > 0 || half > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
-            mma_ts(o_tmem, p_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
-          }
-        }
-        ++n_pv[i];
-        return true;
+      // Each issuer releases every ring block once: a commit after its MMAs
+      // that read the block, or a plain arrive when its query tile did not use
+      // the key tile. Either comes after the block has landed, so it cannot
+      // count toward an earlier fill of the same slot.
+      auto release = [&](uint32_t seq, bool used) {
+        if (used)
+          mma_commit(&ring_empty[seq % kRing]);
+        else
+          mbar_arrive(&ring_empty[seq % kRing]);
       };
-      auto release_v = [&](uint32_t base) {
-        mma_commit(&ring_empty[(base + 3) % kRing]);
-        mma_commit(&ring_empty[(base + 4) % kRing]);
+      // O += P V for the previous key tile, then release its two V blocks.
+      auto finish_prev = [&]() -> bool {
+        if (!wait_block(prev_base + 3, 12) || !wait_block(prev_base + 4, 12)) return false;
+        if (prev_act) {
+          if (!mbar_wait(&p_full[qi], n_pv & 1u, ctl, 11)) return false;
+          tc_fence_after();
+          // Each V block holds 64 keys x 128 value dims, MN-major: value dims
+          // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB
+          // apart (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t vb = block_addr(prev_base + 3 + half);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (n_pv > 0 || half > 0 || kk > 0) ? 1u : 0u;
+              const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
+              mma_ts(o_tmem, s_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
+            }
+          }
+          ++n_pv;
+          issued_any = true;
+        }
+        release(prev_base + 3, prev_act);
+        release(prev_base + 4, prev_act);
+        return true;
       };
 
       uint32_t base = 0;
       for (int kt = tiles.first(); ok && kt < tiles.end;
-           kt = tiles.next(kt), base += kBlocksPerTile) {
-        const bool act[2] = {tiles.active(0, kt), tiles.active(1, kt)};
-        const uint32_t k_addr[3] = {block_addr(base), block_addr(base + 1),
-                                    block_addr(base + 2)};
-        bool k_ready = false;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          if (prev >= 0 && prev_act[i]) {
-            if (!issue_pv(i, prev_base)) { ok = false; break; }
-            issued_any = true;
-          }
-          if (act[i]) {
-            // K is waited for only now, after the previous tile's first PV:
-            // its slots free up late in the previous iteration.
-            if (!k_ready) {
-              if (!wait_block(base, 13) || !wait_block(base + 1, 13) ||
-                  !wait_block(base + 2, 13)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_ready = true;
-            }
-            const uint32_t sQ = smem_u32(smem + kOffQ + i * kQBytes);
-            const uint32_t s_tmem = tmem_base + kColS + 128 * i;
-#pragma unroll
-            for (int blk = 0; blk < 3; ++blk) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
-                const uint64_t kd = sdesc_sw128(k_addr[blk] + kk * 32, 16, 1024);
-                mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
-              }
-            }
-            issued_any = true;
-            mma_commit(&s_full[i]);
+           kt = tiles.next(kt), base += kBlocksPerTile, ++n_tiles) {
+        const bool act = tiles.active(qi, kt);
+        if (prev >= 0 && !finish_prev()) { ok = false; break; }
+        if (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13)) {
+          ok = false;
+          break;
+        }
+        // S order: tile 1 waits for tile 0's S of this key tile, tile 0 for
+        // tile 1's S of the previous one.
+        if (pair) {
+          if (qi == 1) {
+            if (!mbar_wait(&s_issued[0], n_tiles & 1u, ctl, 15)) { ok = false; break; }
+          } else if (n_tiles > 0) {
+            if (!mbar_wait(&s_issued[1], (n_tiles - 1) & 1u, ctl, 15)) { ok = false; break; }
           }
         }
-        if (!ok) break;
-        if (prev >= 0) release_v(prev_base);
-        mma_commit(&ring_empty[base % kRing]);
-        mma_commit(&ring_empty[(base + 1) % kRing]);
-        mma_commit(&ring_empty[(base + 2) % kRing]);
+        if (act) {
+          tc_fence_after();
+          const uint32_t k_addr[3] = {block_addr(base), block_addr(base + 1),
+                                      block_addr(base + 2)};
+#pragma unroll
+          for (int blk = 0; blk < 3; ++blk) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
+              const uint64_t kd = sdesc_sw128(k_addr[blk] + kk * 32, 16, 1024);
+              mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
+            }
+          }
+          issued_any = true;
+          mma_commit(&s_full[qi]);
+        }
+        if (pair) mbar_arrive(&s_issued[qi]);
+        release(base, act);
+        release(base + 1, act);
+        release(base + 2, act);
         prev = kt;
-        prev_act[0] = act[0];
-        prev_act[1] = act[1];
+        prev_act = act;
         prev_base = base;
-        prev_v_ready = false;
       }
-      if (ok && prev >= 0) {
-        for (int i = 0; i < 2 && ok; ++i)
-          if (prev_act[i]) ok = issue_pv(i, prev_base);
-        if (ok) {
-          release_v(prev_base);
-          mma_commit(&o_final);
-        }
-      }
+      if (ok && prev >= 0) ok = finish_prev();
+      if (ok && n_pv > 0) mma_commit(&o_final[qi]);
       if (!ok && issued_any) {
-        mma_commit(&drain_bar);
+        mma_commit(&drain_bar[qi]);
         int zero = 0;
         WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
-        mbar_wait(&drain_bar, 0, drain, 14);
+        mbar_wait(&drain_bar[qi], 0, drain, 14);
       }
     }
   }
@@ -535,23 +561,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       float alpha = 1.f;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
       // Causal tiles after the first: one pass against the running max m,
-      // writing P while tracking the tile's largest s*scale - m. Only if that
-      // exceeds the 2^8 headroom is the tile redone exactly below (new max,
-      // O rescaled). The first tile and the masked kernel always take the
-      // exact two-pass route.
+      // writing P (64 keys per store). Every p is then <= 2^8 unless the max
+      // grew by more than the headroom, so a row sum <= 2^8 proves no rescale
+      // is due; otherwise (rare: many keys near the max, or a new max) the
+      // tile's true max is taken and, only if it grew past the headroom, the
+      // tile is redone exactly below (new max, O rescaled). The first tile and
+      // the masked kernel always take the exact two-pass route.
       bool exact = !(causal_fast && n > 0 && m > -INFINITY);
       if (!exact) {
-        float xmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-          if (diag)
-            p_chunk_causal<true, true>(raw + c * 32, c, r, args.scale_log2, m, pk, acc, xmax);
-          else
-            p_chunk_causal<false, true>(raw + c * 32, c, r, args.scale_log2, m, pk, acc, xmax);
-          tmem_st16(lane_base + colS + 16 * c, pk);
+        for (int c2 = 0; c2 < 4; c2 += 2) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
+            if (diag)
+              p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph, acc);
+            else
+              p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph,
+                                    acc);
+          }
+          tmem_st32(lane_base + colS + 16 * c2, pk);
         }
-        exact = __any_sync(0xffffffffu, fmaxf(xmax[0], xmax[1]) > kRescaleThreshold);
+        const float s_fast = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
+                             ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        bool grew = false;
+        if (__any_sync(0xffffffffu, !(s_fast <= 256.f))) {
+          const float mt = (diag ? raw_row_max<true>(raw, r) : raw_row_max<false>(raw, r)) *
+                           args.scale_log2;
+          grew = mt > m + kRescaleThreshold;
+        }
+        exact = __any_sync(0xffffffffu, grew);
         if (exact) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -642,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]
-    const bool have = ok && n > 0 && mbar_wait_warp(&o_final, 0, ctl, 22);
+    const bool have = ok && n > 0 && mbar_wait_warp(&o_final[wi], 0, ctl, 22);
     if (have) tc_fence_after();
     if (n == 0 || have) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
