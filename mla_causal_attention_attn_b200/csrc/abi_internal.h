@@ -23,6 +23,9 @@ unsigned int* device_error_word();
 // Per-wait limit of the kernels' bounded waits (MLA_WAIT_LIMIT_NS, else 1 s).
 unsigned long long wait_limit_ns();
 
+// 1 when MLA_TEST_STALL_WAIT=1 (failure-detection tests only), else 0.
+int test_stall_wait();
+
 bool aligned16(const void* p);
 size_t round_up(size_t x, size_t a);
 

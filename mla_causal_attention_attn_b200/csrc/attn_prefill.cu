@@ -78,6 +78,7 @@ struct AttnArgs {
   float scale_log2;            // softmax_scale * log2(e)
   unsigned long long wait_limit_ns;
   unsigned int* err_word;      // device status word
+  int test_stall;              // failure-detection test: one wait that never completes
 };
 
 // Which key tiles the two query tiles of a CTA visit. Causal: tile qt visits
@@ -252,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t o_final[2];
   __shared__ uint64_t drain_bar[2];
   __shared__ uint64_t s_issued[2];  // issuer i has issued (or skipped) S of its next tile
+  __shared__ uint64_t never_bar;    // no thread ever arrives (failure-detection test)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -301,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_final[i], 1);
       mbar_init(&drain_bar[i], 1);
       mbar_init(&s_issued[i], 1);
+      mbar_init(&never_bar, 1);
     }
     fence_barrier_init();
   }
@@ -537,6 +540,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) {
       if (!tiles.active(wi, kt)) continue;
       const int k0 = kt * kBKV;
+      // Failure-detection test: query tile 0 of the first CTA waits on a
+      // barrier nothing arrives on; the bounded wait must time out, abort the
+      // CTA cleanly and report through the status word.
+      if (args.test_stall && wi == 0 && blockIdx.x == 0 &&
+          !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
+        ok = false;
+        break;
+      }
       if (!mbar_wait_warp(&s_full[wi], n & 1u, ctl, 20)) { ok = false; break; }
       tc_fence_after();
       // The 128 scores of this thread's row are read from tensor memory once
@@ -801,7 +812,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
-                                cudaStream_t stream) {
+                                int test_stall, cudaStream_t stream) {
   CUtensorMap tmQn, tmQp, tmKn, tmKp, tmV;
   const int BH = B * kH;
   if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
@@ -827,6 +838,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   a.scale_log2 = softmax_scale * kLog2e;
   a.wait_limit_ns = wait_limit_ns;
   a.err_word = err_word;
+  a.test_stall = test_stall;
   const long long ctas = (long long)B * kH * a.n_pairs;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
   kern<<<unsigned(ctas), kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, a);

@@ -29,6 +29,6 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
-                                cudaStream_t stream);
+                                int test_stall, cudaStream_t stream);
 
 }  // namespace mla

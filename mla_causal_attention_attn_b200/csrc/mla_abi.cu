@@ -49,6 +49,18 @@ unsigned long long wait_limit_ns() {
   return v;
 }
 
+// MLA_TEST_STALL_WAIT=1 (read once) makes the attention kernel's first CTA
+// wait on a barrier that nothing completes, so that tests can check that the
+// bounded wait gives up, the CTA aborts cleanly and MLA_ERR_TIMEOUT is
+// reported. Never set in normal use.
+int test_stall_wait() {
+  static const int v = [] {
+    const char* s = std::getenv("MLA_TEST_STALL_WAIT");
+    return (s && s[0] == '1' && s[1] == '\0') ? 1 : 0;
+  }();
+  return v;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -87,7 +99,8 @@ mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_n
   }
   return from_cuda(launch_attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld,
                                        mask ? cls : nullptr, B, T, softmax_scale, out,
-                                       wait_limit_ns(), device_error_word(), stream));
+                                       wait_limit_ns(), device_error_word(), test_stall_wait(),
+                                       stream));
 }
 
 }  // namespace abi

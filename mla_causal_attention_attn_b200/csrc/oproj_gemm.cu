@@ -23,7 +23,10 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kGroupM = 16;
+// Output tiles are visited in groups of kGroupM row blocks (all column
+// blocks of a group before the next): for M = 4096 the whole A (64 MiB) stays
+// in L2 while W_o streams through once.
+constexpr int kGroupM = 32;
 constexpr int kThreads = 192;
 
 __device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
@@ -42,9 +45,11 @@ struct GemmCfg {
   static constexpr uint32_t kABytes = kBM * kBK * 2;
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+  // two accumulators, rounded up to the power-of-two allocation granule
+  static constexpr uint32_t kTmemCols = 2 * BN <= 128 ? 128u : (2 * BN <= 256 ? 256u : 512u);
   static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
-  static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
+  static_assert(BN == 64 || BN == 128 || BN == 224 || BN == 256, "BN");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "TMEM columns must be a power of two in [32, 512]");
 };
@@ -258,16 +263,32 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, i
 }  // namespace
 
 int oproj_pick_bn(int64_t M, int N, int num_sms) {
+  // Largest expected throughput: fraction of the last wave's SMs kept busy,
+  // times a per-tile efficiency of the narrower MMAs (measured on B200: an
+  // M128 N64 MMA runs at ~0.7 of the N128/N256 rate per FLOP).
   const int64_t m_tiles = (M + kBM - 1) / kBM;
-  if (m_tiles * (N / 256) >= num_sms) return 256;
-  if (m_tiles * (N / 128) >= num_sms) return 128;
-  return 64;
+  const int cand[4] = {256, 224, 128, 64};
+  const double tile_eff[4] = {1.0, 0.985, 0.95, 0.7};
+  int best = 64;
+  double best_score = -1.0;
+  for (int i = 0; i < 4; ++i) {
+    const int bn = cand[i];
+    if (N % bn != 0) continue;
+    const int64_t tiles = m_tiles * (N / bn);
+    const int64_t waves = (tiles + num_sms - 1) / num_sms;
+    const double score = double(tiles) / double(waves * num_sms) * tile_eff[i];
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = bn;
+    }
+  }
+  return best;
 }
 
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
                               unsigned int* err_word, cudaStream_t stream) {
-  if (M <= 0 || N % 256 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
+  if (M <= 0 || N % 64 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
     return cudaErrorInvalidValue;
   CUtensorMap tmA;
   const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
@@ -275,10 +296,14 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
   const uint32_t box[2] = {kBK, kBM};
   if (!encode_tmap_bf16(&tmA, A, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
   const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
+  if (N % bn != 0) return cudaErrorInvalidValue;
   auto* Cb = static_cast<__nv_bfloat16*>(C);
   switch (bn) {
     case 256:
       return launch_bn<256, 4>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+                                 stream);
+    case 224:
+      return launch_bn<224, 5>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
                                  stream);
     case 128:
       return launch_bn<128, 6>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,

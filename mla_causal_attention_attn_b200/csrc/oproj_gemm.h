@@ -7,8 +7,9 @@
 namespace mla {
 
 // C[M, N] = A[M, K] . W[N, K]^T, all bf16 row-major, fp32 accumulation.
-// Requires N % 256 == 0, K % 64 == 0, 16-byte aligned pointers. `force_bn`
-// (0, 64, 128 or 256) overrides the tile-width choice.
+// Requires N % 64 == 0, K % 64 == 0, 16-byte aligned pointers; the tile width
+// BN (64, 128, 224 or 256, dividing N) is chosen for wave efficiency unless
+// `force_bn` (non-zero) fixes it.
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
                               unsigned int* err_word, cudaStream_t stream);
