@@ -251,8 +251,10 @@ def workload_config(w, flushed=True):
     return {
         "workload": w.name, "B": w.B, "T": w.T, "heads": H,
         "qk_head_dim": "128 nope + 64 rope (rope key shared by all heads)", "v_head_dim": DV,
-        "o_proj": "8192 -> 7168", "mask": "causal + key padding [B,1,T,T]" if w.key_padding
-        else "causal (implicit)", "q_scale": w.q_scale,
+        "o_proj": "8192 -> 7168",
+        "mask": ("causal + key padding as valid lengths [B]" if w.compact_mask
+                 else "causal + key padding [B,1,T,T]") if w.key_padding else "causal (implicit)",
+        "q_scale": w.q_scale,
         "l2": "flushed between timed steps (256 MiB write, outside the step events)"
         if flushed else "n/a",
         "parallelism": "independent batch per GPU (no collective)",
@@ -268,11 +270,16 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.set_device(dev)
     binding.load()
     d = inputs.make_workload(w, seed=rank)
-    names = ["q_nope", "q_pe", "k_nope", "k_pe", "v"] + (["mask"] if d["mask"] is not None else [])
+    compact = w.compact_mask
+    if compact:
+        d["valid_len_i32"] = d["valid_len"].to(torch.int32)
+    extra = ["valid_len_i32"] if compact else (["mask"] if d["mask"] is not None else [])
+    names = ["q_nope", "q_pe", "k_nope", "k_pe", "v"] + extra
     g = {k: d[k].to(dev) for k in names}
     W = d["W_o"].to(dev)
     B, T = w.B, w.T
-    ws_attn = torch.empty(binding.attn_prefill_workspace_bytes(B, T, d["mask"] is not None) or 16,
+    dense_mask = d["mask"] is not None and not compact
+    ws_attn = torch.empty(binding.attn_prefill_workspace_bytes(B, T, dense_mask) or 16,
                           dtype=torch.uint8, device=dev)
     attn = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=dev)
     out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=dev)
@@ -283,9 +290,14 @@ def run_ours(args, w, rank, world, local_rank):
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
-                             mask=g.get("mask"), softmax_scale=scale, out=attn,
-                             workspace=ws_attn, stream=stream)
+        if compact:
+            binding.attn_prefill_varlen(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                        g["valid_len_i32"], softmax_scale=scale, out=attn,
+                                        stream=stream)
+        else:
+            binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                 mask=g.get("mask"), softmax_scale=scale, out=attn,
+                                 workspace=ws_attn, stream=stream)
         if ev:
             ev[1].record(stream)
         binding.o_proj(attn, W, out=out, stream=stream)
@@ -337,7 +349,7 @@ def run_ours(args, w, rank, world, local_rank):
     if not args.no_e2e:
         host = {k: d[k].pin_memory() for k in names}
         out_h = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16).pin_memory()
-        ws_f = torch.empty(binding.attn_oproj_workspace_bytes(B, T, d["mask"] is not None),
+        ws_f = torch.empty(binding.attn_oproj_workspace_bytes(B, T, dense_mask),
                            dtype=torch.uint8, device=dev)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = out_h.numel() * out_h.element_size()
@@ -346,9 +358,14 @@ def run_ours(args, w, rank, world, local_rank):
         def e2e_step():
             for k in names:
                 g[k].copy_(host[k], non_blocking=True)
-            binding.attn_oproj(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"], W,
-                               mask=g.get("mask"), softmax_scale=scale, out=out,
-                               workspace=ws_f, stream=stream)
+            if compact:
+                binding.attn_oproj_varlen(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                          g["valid_len_i32"], W, softmax_scale=scale, out=out,
+                                          workspace=ws_f, stream=stream)
+            else:
+                binding.attn_oproj(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"], W,
+                                   mask=g.get("mask"), softmax_scale=scale, out=out,
+                                   workspace=ws_f, stream=stream)
             out_h.copy_(out, non_blocking=True)
 
         e2e_step()
@@ -365,9 +382,10 @@ def run_ours(args, w, rank, world, local_rank):
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": job_tflops(world, flops_step, n_e2e, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
-               "ms_per_step": e2e_ms / n_e2e, "call": "mla_attn_oproj",
-               "note": "per step: pinned H2D of the activations (and mask), the fused call, "
-                       "D2H of the output; W_o resident like any weight"}
+               "ms_per_step": e2e_ms / n_e2e,
+               "call": "mla_attn_oproj_varlen" if compact else "mla_attn_oproj",
+               "note": "per step: pinned H2D of the activations (and mask or valid lengths), "
+                       "the fused call, D2H of the output; W_o resident like any weight"}
 
     if rank != 0:
         return
@@ -404,7 +422,7 @@ def run_ours(args, w, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
-        "gpu_launches": args.steps * (2 + (1 if d["mask"] is not None else 0)),
+        "gpu_launches": args.steps * (2 + (1 if dense_mask else 0)),
         "wall_s_timed_region": wall,
     }
     print(json.dumps(line), flush=True)

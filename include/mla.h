@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 1
+#define MLA_ABI_VERSION 2
 
 /* Model dimensions (fixed at compile time; no other values are accepted). */
 #define MLA_NUM_HEADS 64
@@ -141,6 +141,36 @@ mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
                             const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
                             int T, float softmax_scale, const mla_bf16* W_o, void* workspace,
                             size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
+
+/*
+ * Causal attention with key padding given compactly, as one valid length per
+ * sequence instead of a [B,1,T,T] mask (page "Kimi K2 · Transformer blocks",
+ * excerpt modeling_deepseek.py 1443-1457: the flash path keeps the 2-D padding
+ * mask, the other paths expand it with the causal mask into the 4-D additive
+ * form). For right-padded sequences the two forms agree: key j is allowed for
+ * query i iff j <= i and j < valid_len[b]. Query rows i >= valid_len[b] still
+ * attend to the sequence's valid keys and are written like any other row.
+ *
+ *   valid_len  device array of B int32 (4-byte aligned), read by the kernel;
+ *              values are clamped to [0, T]. A sequence with valid_len 0 has
+ *              no allowed key: its rows are zeros.
+ * Every other argument as in mla_attn_prefill with mask == NULL (no workspace
+ * is needed). NULL valid_len -> MLA_ERR_INVALID_ARG.
+ */
+mla_status_t mla_attn_prefill_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                     const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                     const mla_bf16* v, const int32_t* valid_len, int B, int T,
+                                     float softmax_scale, mla_bf16* out, mla_stream_t stream);
+
+/*
+ * mla_attn_prefill_varlen followed by o_proj, as mla_attn_oproj; workspace of
+ * mla_attn_oproj_workspace_bytes(B, T, 0) bytes.
+ */
+mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                   const mla_bf16* v, const int32_t* valid_len, int B, int T,
+                                   float softmax_scale, const mla_bf16* W_o, void* workspace,
+                                   size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
 
 /* Largest B*T mla_attn_oproj_noalloc accepts (its fixed scratch holds the
  * merged attention output of this many tokens: 64 MiB). */

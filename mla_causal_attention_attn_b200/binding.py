@@ -49,6 +49,11 @@ _SIGNATURES = {
     "mla_attn_oproj_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_float, _VP,
                                               _VP, _VP]),
+    "mla_attn_prefill_varlen": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_float, _VP, _VP]),
+    "mla_attn_oproj_varlen": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_float, _VP, _VP,
+                                             ctypes.c_size_t, _VP, _VP]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_abi_version": (ctypes.c_int, []),
@@ -196,6 +201,65 @@ def attn_oproj(q_nope, q_pe, k_nope, k_pe, v, W_o, mask=None, softmax_scale=None
                             _ptr(mask), mask_ld, B, T, scale, _ptr(W_o), _ptr(workspace),
                             ws_bytes, _ptr(out), _stream_handle(stream))
     _check("mla_attn_oproj", st)
+    return out
+
+
+def _valid_len(valid_len, B):
+    if valid_len.dtype != torch.int32 or not valid_len.is_cuda:
+        raise TypeError("valid_len must be an int32 CUDA tensor")
+    if tuple(valid_len.shape) != (B,) or not valid_len.is_contiguous():
+        raise ValueError(f"valid_len must be a contiguous [{B}] tensor")
+    return valid_len
+
+
+def attn_prefill_varlen(q_nope, q_pe, k_nope, k_pe, v, valid_len, softmax_scale=None, out=None,
+                        stream=None):
+    """Causal attention with key padding (keys j >= valid_len[b] excluded),
+    [B, T, 8192] bf16, via ``mla_attn_prefill_varlen``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _valid_len(valid_len, B)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, K_OPROJ), "out")
+    st = lib.mla_attn_prefill_varlen(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                     _ptr(valid_len), B, T, scale, _ptr(out),
+                                     _stream_handle(stream))
+    _check("mla_attn_prefill_varlen", st)
+    return out
+
+
+def attn_oproj_varlen(q_nope, q_pe, k_nope, k_pe, v, valid_len, W_o, softmax_scale=None,
+                      out=None, workspace=None, stream=None):
+    """Whole path with key padding given as valid lengths, [B, T, 7168] bf16,
+    via ``mla_attn_oproj_varlen``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    _valid_len(valid_len, B)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    need = attn_oproj_workspace_bytes(B, T, False)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.mla_attn_oproj_varlen(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                   _ptr(valid_len), B, T, scale, _ptr(W_o), _ptr(workspace),
+                                   ws_bytes, _ptr(out), _stream_handle(stream))
+    _check("mla_attn_oproj_varlen", st)
     return out
 
 

@@ -40,11 +40,12 @@ mla_status_t check_attn_args(const void* q_nope, const void* q_pe, const void* k
 mla_status_t from_cuda(cudaError_t e);
 
 // Mask-tile classification (when mask is given, into `cls`) followed by the
-// attention kernel writing the merged heads to `out`.
+// attention kernel writing the merged heads to `out`. valid_len (device [B],
+// only without mask) selects causal attention with key padding.
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
-                           cudaStream_t stream);
+                           cudaStream_t stream, const int* valid_len = nullptr);
 
 }  // namespace abi
 }  // namespace mla

@@ -8,6 +8,10 @@
 //     out[b, i, h*128 + e] = sum_j p_ij v_je
 //   with k_pe one [B,1,T,64] tensor shared by all heads and M either the
 //   implicit causal mask (mask == NULL) or an explicit additive [B,1,T,T] mask.
+//   The causal kernel also takes the compact form of causal + key padding
+//   (page "Kimi K2 · Transformer blocks", excerpt modeling_deepseek.py
+//   1443-1457: the 2-D padding mask of the flash path): key j is allowed for
+//   query i iff j <= i and j < valid_len[b].
 //
 // One CTA computes two 128-row query tiles (2p, 2p+1) of one (b, h), so that
 // every K/V tile brought into shared memory serves 256 query rows and the
@@ -70,6 +74,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 struct AttnArgs {
   const __nv_bfloat16* mask;   // [B,1,T,mask_ld] or null (causal)
+  const int* valid_len;        // [B] keys per sequence (causal kernel), or null (all T)
   int64_t mask_ld;
   int mask_vec;                // rows 16-byte aligned: vector loads
   const uint8_t* tile_class;   // [B, n_qt, n_kv] or null
@@ -82,19 +87,21 @@ struct AttnArgs {
 };
 
 // Which key tiles the two query tiles of a CTA visit. Causal: tile qt visits
-// 0..qt. Explicit mask: every key tile whose class is not "all -inf" (every
-// tile when no classification is given).
+// 0..qt, and none at or past the sequence's key count (kv_end tiles). Explicit
+// mask: every key tile whose class is not "all -inf" (every tile when no
+// classification is given).
 template <bool kMasked>
 struct PairTiles {
   int qt[2];
   bool exists[2];
   const uint8_t* cls[2];
-  int end;  // one past the last candidate key tile
+  int kv_end;  // causal: key tiles holding at least one of the sequence's keys
+  int end;     // one past the last candidate key tile
 
   __device__ __forceinline__ bool active(int i, int kt) const {
     if (!exists[i]) return false;
     if (kMasked) return cls[i] ? cls[i][kt] != kTileSkip : true;
-    return kt <= qt[i];
+    return kt <= qt[i] && kt < kv_end;
   }
   __device__ __forceinline__ int next(int kt) const {
     ++kt;
@@ -272,6 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = (grp % (kH / kHeadGroup)) * kHeadGroup + rem % kHeadGroup;
   const int pair = args.n_pairs - 1 - rem / kHeadGroup;
   const int bh = b * kH + h;
+  // Keys of this sequence: T, or valid_len[b] clamped to [0, T].
+  const int n_keys =
+      (!kMasked && args.valid_len) ? min(max(args.valid_len[b], 0), args.T) : args.T;
 
   PairTiles<kMasked> tiles;
 #pragma unroll
@@ -282,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        ? args.tile_class + (size_t(b) * args.n_qt + tiles.qt[i]) * args.n_kv
                        : nullptr;
   }
-  tiles.end = kMasked ? args.n_kv : min(2 * pair + 2, args.n_qt);
+  tiles.kv_end = (n_keys + kBKV - 1) / kBKV;
+  tiles.end = kMasked ? args.n_kv : min(min(2 * pair + 2, args.n_qt), tiles.kv_end);
   const bool has_work = tiles.first() < tiles.end;
 
   WaitCtl ctl{&abort_flag, args.wait_limit_ns, kErrKernelAttn, args.err_word};
@@ -560,9 +571,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
       sc.kvalid = args.T - k0;
       sc.mask_vec = args.mask_vec;
-      sc.diag_row = (!kMasked && kt == qt) ? r : kBKV;  // causal: key c allowed iff c <= r
+      // Causal kernel: keys c <= lim of the tile are allowed (c <= r on the
+      // query tile's own key tile, and none at or past the sequence's key
+      // count). `diag` marks the tiles where that limit cuts (warp-uniform).
+      const bool diag = !kMasked && (kt == qt || n_keys - k0 < kBKV);
+      const int lim = min(kt == qt ? r : kBKV - 1, n_keys - 1 - k0);
+      sc.diag_row = diag ? lim : kBKV;
       const bool causal_fast = !kMasked && args.scale_log2 > 0.f;
-      const bool diag = !kMasked && kt == qt;
       uint32_t raw[kBKV];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -587,7 +602,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int h2 = 0; h2 < 2; ++h2) {
             uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
             if (diag)
-              p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph, acc);
+              p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, lim, args.scale_log2, m, ph,
+                                   acc);
             else
               p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph,
                                     acc);
@@ -598,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         bool grew = false;
         if (__any_sync(0xffffffffu, !(s_fast <= 256.f))) {
-          const float mt = (diag ? raw_row_max<true>(raw, r) : raw_row_max<false>(raw, r)) *
+          const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
                            args.scale_log2;
           grew = mt > m + kRescaleThreshold;
         }
@@ -613,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (causal_fast) {
         // positive scale: the maximum of the raw scores gives the maximum of
         // the scaled ones
-        mt = diag ? raw_row_max<true>(raw, r) : raw_row_max<false>(raw, r);
+        mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
         mt *= args.scale_log2;
       } else {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -649,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
         if (causal_fast) {
           if (diag)
-            p_chunk_causal<true>(rc, c, r, args.scale_log2, m_use, pk, acc);
+            p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
           else
             p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
         } else {
@@ -812,7 +828,8 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
-                                int test_stall, cudaStream_t stream) {
+                                int test_stall, cudaStream_t stream, const int* valid_len) {
+  if (mask && valid_len) return cudaErrorInvalidValue;
   CUtensorMap tmQn, tmQp, tmKn, tmKp, tmV;
   const int BH = B * kH;
   if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
@@ -827,6 +844,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   AttnArgs a;
   a.mask = static_cast<const __nv_bfloat16*>(mask);
   a.mask_ld = mask_ld;
+  a.valid_len = valid_len;
   a.mask_vec = mask_rows_vec_ok(mask, mask_ld) ? 1 : 0;
   a.tile_class = static_cast<const uint8_t*>(tile_class);
   a.out = static_cast<__nv_bfloat16*>(out);

@@ -23,12 +23,15 @@ cudaError_t launch_mask_classify(const void* mask, int64_t mask_ld, int B, int T
 
 // Prefill attention for all 64 heads; writes out[b, t, h*128 + e] (bf16).
 // mask == null: causal. tile_class may be null when mask is given (every key
-// tile is then visited and masked element-wise).
+// tile is then visited and masked element-wise). valid_len (device, [B] int32,
+// only without mask): causal with keys j >= valid_len[b] masked (values are
+// clamped to [0, T]); null means every sequence has all T keys.
 cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void* k_nope,
                                 const void* k_pe, const void* v, const void* mask,
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
-                                int test_stall, cudaStream_t stream);
+                                int test_stall, cudaStream_t stream,
+                                const int* valid_len = nullptr);
 
 }  // namespace mla

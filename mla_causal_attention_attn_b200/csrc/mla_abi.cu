@@ -92,7 +92,7 @@ mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, const int* valid_len) {
   if (mask) {
     mla_status_t s = from_cuda(launch_mask_classify(mask, mask_ld, B, T, cls, stream));
     if (s != MLA_OK) return s;
@@ -100,7 +100,7 @@ mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_n
   return from_cuda(launch_attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld,
                                        mask ? cls : nullptr, B, T, softmax_scale, out,
                                        wait_limit_ns(), device_error_word(), test_stall_wait(),
-                                       stream));
+                                       stream, valid_len));
 }
 
 }  // namespace abi
@@ -178,6 +178,47 @@ mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
                     attn, st);
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, device_error_word(),
+                                     st));
+}
+
+mla_status_t mla_attn_prefill_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                     const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                     const mla_bf16* v, const int32_t* valid_len, int B, int T,
+                                     float softmax_scale, mla_bf16* out, mla_stream_t stream) {
+  if (!valid_len) return MLA_ERR_INVALID_ARG;
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(valid_len) & 3u) != 0) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  return run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale,
+                       nullptr, out, reinterpret_cast<cudaStream_t>(stream), valid_len);
+}
+
+mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                   const mla_bf16* v, const int32_t* valid_len, int B, int T,
+                                   float softmax_scale, const mla_bf16* W_o, void* workspace,
+                                   size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  if (!valid_len || !W_o) return MLA_ERR_INVALID_ARG;
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if ((reinterpret_cast<uintptr_t>(valid_len) & 3u) != 0 || !aligned16(W_o))
+    return MLA_ERR_MISALIGNED;
+  if (int64_t(B) * int64_t(T) > kMaxM) return MLA_ERR_SHAPE;
+  const size_t need = mla_attn_oproj_workspace_bytes(B, T, 0);
+  if (!workspace || workspace_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale, nullptr,
+                    workspace, st, valid_len);
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(workspace, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
                                      device_sm_count(), wait_limit_ns(), 0, device_error_word(),
                                      st));
 }

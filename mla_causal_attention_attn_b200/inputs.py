@@ -42,6 +42,7 @@ class Workload:
     q_scale: float = 1.0
     key_padding: bool = False
     min_valid: int = 512
+    compact_mask: bool = False  # key padding passed as valid lengths, not the dense mask
 
     @property
     def tokens(self) -> int:
@@ -55,6 +56,9 @@ WORKLOADS = {
     "b16_t1024_causal": Workload("b16_t1024_causal", 16, 1024),
     "b1_t32768_causal_qx2": Workload("b1_t32768_causal_qx2", 1, 32768, q_scale=2.0),
     "b8_t4096_keypad_mask": Workload("b8_t4096_keypad_mask", 8, 4096, key_padding=True),
+    # the same inputs, the padding given as per-sequence valid lengths
+    "b8_t4096_keypad_varlen": Workload("b8_t4096_keypad_varlen", 8, 4096, key_padding=True,
+                                       compact_mask=True),
 }
 
 

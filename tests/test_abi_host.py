@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 1
+    assert lib.mla_abi_version() == 2
     for code, name in binding.STATUS.items():
         assert lib.mla_status_string(code).decode() == name
     assert lib.mla_status_string(12345).decode() == "MLA_ERR_UNKNOWN"
@@ -119,12 +119,39 @@ def test_fused_argument_errors(lib):
     assert fused(lib, mask=A, ld=64, ws_bytes=64 * 8192 * 2) == WORKSPACE  # class bytes missing
 
 
+def varlen(lib, q=A, qp=A, k=A, kp=A, v=A, vl=A, B=1, T=64, scale=0.07, out=A):
+    return lib.mla_attn_prefill_varlen(q, qp, k, kp, v, vl, B, T, scale, out, None)
+
+
+def fused_varlen(lib, q=A, qp=A, k=A, kp=A, v=A, vl=A, B=1, T=64, scale=0.07, W=A, ws=A,
+                 ws_bytes=1 << 40, out=A):
+    return lib.mla_attn_oproj_varlen(q, qp, k, kp, v, vl, B, T, scale, W, ws, ws_bytes, out, None)
+
+
+def test_varlen_argument_errors(lib):
+    assert varlen(lib, vl=None) == INVALID
+    assert varlen(lib, q=None) == INVALID
+    assert varlen(lib, scale=float("nan")) == INVALID
+    assert varlen(lib, B=0) == SHAPE
+    assert varlen(lib, T=0) == SHAPE
+    assert varlen(lib, vl=A + 2) == MISALIGNED  # int32 array must be 4-byte aligned
+    assert varlen(lib, k=A + 8) == MISALIGNED
+    assert fused_varlen(lib, vl=None) == INVALID
+    assert fused_varlen(lib, W=None) == INVALID
+    assert fused_varlen(lib, W=A + 2) == MISALIGNED
+    assert fused_varlen(lib, vl=A + 1) == MISALIGNED
+    assert fused_varlen(lib, ws=None) == WORKSPACE
+    assert fused_varlen(lib, ws_bytes=64 * 8192 * 2 - 1) == WORKSPACE
+    assert fused_varlen(lib, ws=A + 8) == MISALIGNED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path only")
 def test_valid_call_without_device_reports_cuda_error(lib):
     """With no usable device a well-formed call fails cleanly (MLA_ERR_CUDA)
     instead of launching anything."""
     assert prefill(lib) in (CUDA, UNSUPPORTED)
     assert lib.mla_o_proj(A, A, 4, A, None) in (CUDA, UNSUPPORTED)
+    assert varlen(lib) in (CUDA, UNSUPPORTED)
 
 
 def test_binding_refuses_missing_library(tmp_path):
