@@ -42,6 +42,8 @@ DEFAULT_WORKLOAD = "b1_t4096_causal"
 H, DQK, DV, D_MODEL, K_OPROJ = 64, 192, 128, 7168, 8192
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DATASHEET_BF16_TFLOPS = 2250.0
+# Timed regions at least this long run into the power cap (sustained peak).
+LONG_REGION_S = 0.5
 
 
 # ---------------------------------------------------------------- FLOP counts
@@ -397,10 +399,19 @@ def run_ours(args, w, rank, world, local_rank):
     dom = max(kern, key=lambda k: kern[k][1])
     f_dom, t_dom, src_dom, kname = kern[dom]
     achieved = f_dom / (t_dom * 1e-3) / 1e12
+    # A kernel timed inside a long loop runs under the power cap: its
+    # denominator is the sustained GEMM peak; a short timed region gets the
+    # burst peak. Both fractions are reported.
+    long_region = wall >= LONG_REGION_S
+    peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
     roofline = {"kernel": kname, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"],
-                "peak_source": f"{peak_src} bf16 burst",
+                "peak": peaks[peak_key], "unit": "TFLOP/s",
+                "frac": achieved / peaks[peak_key],
+                "peak_source": f"{peak_src} bf16 " + (
+                    f"sustained (timed region {wall:.2f} s)" if long_region
+                    else f"burst (timed region {wall:.2f} s)"),
+                "frac_of_burst": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": recorded_traffic(src_dom, w.name),
                 "per_launch_flops": f_dom, "avg_launch_ms": t_dom}
     cpu = None

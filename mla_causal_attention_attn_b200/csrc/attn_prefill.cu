@@ -592,8 +592,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // is due; otherwise (rare: many keys near the max, or a new max) the
       // tile's true max is taken and, only if it grew past the headroom, the
       // tile is redone exactly below (new max, O rescaled). The first tile and
-      // the masked kernel always take the exact two-pass route.
-      bool exact = !(causal_fast && n > 0 && m > -INFINITY);
+      // the masked kernel always take the exact two-pass route. The choice is
+      // warp-uniform (a row whose max is still -inf fails the row-sum test).
+      bool exact = !(causal_fast && n > 0);
+      float rowsum = 0.f;
       if (!exact) {
 #pragma unroll
         for (int c2 = 0; c2 < 4; c2 += 2) {
@@ -610,18 +612,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st32(lane_base + colS + 16 * c2, pk);
         }
-        const float s_fast = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
-                             ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        bool grew = false;
-        if (__any_sync(0xffffffffu, !(s_fast <= 256.f))) {
+        rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        if (__any_sync(0xffffffffu, !(rowsum <= 256.f))) {
           const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
                            args.scale_log2;
-          grew = mt > m + kRescaleThreshold;
-        }
-        exact = __any_sync(0xffffffffu, grew);
-        if (exact) {
+          exact = __any_sync(0xffffffffu, !(mt <= m + kRescaleThreshold));
+          if (exact) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+          }
         }
       }
       if (exact) {
@@ -682,13 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st16(lane_base + colS + 16 * c, pk);
       }
-      }  // exact
-      const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) +
-                           ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 
       // O holds P_{n-1} V_{n-1} here: that PV was issued before this S, and
       // the commit behind s_full covers every earlier MMA. The rescale lands
-      // before PV_n, which waits for p_full below.
+      // before PV_n, which waits for p_full below. (Only the exact route can
+      // change the max.)
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -701,6 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(lane_base + colO + c * 32, rr);
         }
       }
+      }  // exact
       l = l * alpha + rowsum;
       tmem_st_wait();
       tc_fence_before();

@@ -13,6 +13,9 @@
 //     tcgen05.mma (M=128, N=BN, K=16) into one of two TMEM accumulators;
 //   * warps 2..5 drain the finished accumulator (tcgen05.ld), convert to bf16
 //     and store, while the MMA warp already fills the other accumulator.
+// For M <= 128 the product is bound by reading W and runs in
+// oproj_small_m_kernel (below): operands swapped, K split over a cluster of
+// two CTAs, partial sums combined through distributed shared memory.
 #include "oproj_gemm.h"
 #include "host_util.h"
 #include "sm100.cuh"
@@ -29,6 +32,7 @@ constexpr int kBK = 64;
 // (M = 4096 .. 32768, interleaved timing); 16 moved the least DRAM data.
 constexpr int kGroupM = 16;
 constexpr int kThreads = 192;
+constexpr int64_t kSmallMMax = 128;  // M up to this goes to oproj_small_m_kernel
 
 __device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
                                                  int& nb) {
@@ -49,7 +53,7 @@ struct GemmCfg {
   // two accumulators, rounded up to the power-of-two allocation granule
   static constexpr uint32_t kTmemCols = 2 * BN <= 128 ? 128u : (2 * BN <= 256 ? 256u : 512u);
   static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
-  static_assert(BN == 64 || BN == 128 || BN == 224 || BN == 256, "BN");
+  static_assert(BN == 128 || BN == 224 || BN == 256, "BN");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
                 "TMEM columns must be a power of two in [32, 512]");
@@ -261,6 +265,234 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, i
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- small M
+// C[M, N] = A[M, K] . W[N, K]^T for M <= 128, where the product is bound by
+// reading W once from HBM. The operands swap roles: each CTA computes
+// D = W_tile . A^T (M = 128 rows of W, N = NM >= M columns, one per token),
+// so the shared-memory ring holds mostly W and the MMA accumulates
+// C^T[128, NM] in tensor memory. K is split in two halves over the two CTAs
+// of a cluster: the CTA of rank 1 writes its fp32 partial sum into its own
+// (now idle) ring, the CTA of rank 0 adds it through distributed shared
+// memory, rounds to bf16 and stores. Both hand-offs between the two CTAs are
+// mbarriers with bounded waits: part_ready (in rank 0, the partial is written)
+// and part_done (in rank 1, rank 0 has read it; rank 1 keeps its shared
+// memory until then).
+constexpr int kSmallThreads = 192;
+constexpr int kSmallWRows = 128;
+
+template <int NM, int STAGES>
+struct SmallCfg {
+  static constexpr uint32_t kWBytes = kSmallWRows * kBK * 2;  // 16 KB
+  static constexpr uint32_t kABytes = NM * kBK * 2;
+  static constexpr uint32_t kStageBytes = kWBytes + kABytes;
+  static constexpr uint32_t kRowFloats = NM + 4;  // padded partial row (bank spread)
+  static constexpr uint32_t kPartBytes = kSmallWRows * kRowFloats * 4;
+  static constexpr uint32_t kTmemCols = NM;
+  static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
+  static_assert(NM == 32 || NM == 64 || NM == 128, "NM");
+  static_assert(kPartBytes <= STAGES * kStageBytes, "partial fits in the ring");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int NM, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
+    oproj_small_m_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ C,
+                         int M, int N, int K, unsigned long long wait_limit_ns,
+                         unsigned int* err_word) {
+  using Cfg = SmallCfg<NM, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t full_bar[STAGES];
+  __shared__ uint64_t empty_bar[STAGES];
+  __shared__ uint64_t acc_full;
+  __shared__ uint64_t part_ready;  // rank 0: rank 1's partial is in its shared memory
+  __shared__ uint64_t part_done;   // rank 1: rank 0 has read the partial
+  __shared__ uint64_t drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int n0 = int(blockIdx.x >> 1) * kSmallWRows;  // first W row (output column)
+  const int k_blocks = K / kBK / 2;                    // this CTA's half of K
+  const int kb0 = int(rank) * k_blocks;
+
+  WaitCtl ctl{&abort_flag, wait_limit_ns, kErrKernelOprojSmallM, err_word};
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&part_ready, 128);
+    mbar_init(&part_done, 128);
+    mbar_init(&drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  // Both CTAs' barriers are initialised before either can touch the other's.
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmW);
+      uint32_t issued_mask = 0, issued_par = 0;
+      bool ok = true;
+      for (int i = 0; i < k_blocks; ++i) {
+        const int stage = i % STAGES;
+        const uint32_t phase = uint32_t(i / STAGES) & 1u;
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, ctl, 1)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sw = smem + size_t(stage) * Cfg::kStageBytes;
+        uint8_t* sa = sw + Cfg::kWBytes;
+        mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+        tma_load_2d(sw, &tmW, &full_bar[stage], (kb0 + i) * kBK, n0);
+        tma_load_2d(sa, &tmA, &full_bar[stage], (kb0 + i) * kBK, 0);
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+      }
+      if (!ok) {
+        int zero = 0;
+        WaitCtl drain{&zero, wait_limit_ns, kErrKernelOprojSmallM, err_word};
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) mbar_wait(&full_bar[s], (issued_par >> s) & 1u, drain, 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kSmallWRows, NM, false, false);
+      bool ok = true;
+      bool issued_any = false;
+      for (int i = 0; i < k_blocks; ++i) {
+        const int stage = i % STAGES;
+        const uint32_t phase = uint32_t(i / STAGES) & 1u;
+        if (!mbar_wait(&full_bar[stage], phase, ctl, 4)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t w_addr = smem_u32(smem + size_t(stage) * Cfg::kStageBytes);
+        const uint32_t a_addr = w_addr + Cfg::kWBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t wd = sdesc_sw128(w_addr + kk * 32, 16, 1024);
+          const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+          mma_ss(tmem_base, wd, ad, idesc, (i | kk) != 0 ? 1u : 0u);
+        }
+        issued_any = true;
+        mma_commit(&empty_bar[stage]);
+      }
+      if (ok) mma_commit(&acc_full);
+      if (!ok && issued_any) {
+        mma_commit(&drain_bar);
+        int zero = 0;
+        WaitCtl drain{&zero, wait_limit_ns, kErrKernelOprojSmallM, err_word};
+        mbar_wait(&drain_bar, 0, drain, 5);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // Thread = TMEM lane = W row n0 + r; its TMEM columns are the tokens.
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    float* part = reinterpret_cast<float*>(smem);  // rank 1's partial, [128][kRowFloats]
+    if (mbar_wait_warp(&acc_full, 0, ctl, 6)) {
+      tc_fence_after();
+      if (rank == 1) {
+        // All MMAs (the ring's last readers) are done: the ring holds the partial.
+#pragma unroll 1
+        for (int c = 0; c < NM / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem_addr(tmem_base, quad * 32, c * 32), v);
+          tmem_ld_wait();
+          reg_fence(v);
+          float4* dst = reinterpret_cast<float4*>(part + r * Cfg::kRowFloats + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+        mbar_arrive_cluster(mapa_shared(smem_u32(&part_ready), 0));
+        // Keep this CTA's shared memory until rank 0 has read the partial.
+        mbar_wait_cluster(&part_done, 0, ctl, 8);
+      } else if (mbar_wait_cluster(&part_ready, 0, ctl, 7)) {
+        const uint32_t remote = mapa_shared(smem_u32(part + r * Cfg::kRowFloats), 1);
+        const int n = n0 + r;
+#pragma unroll 1
+        for (int c = 0; c < NM / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem_addr(tmem_base, quad * 32, c * 32), v);
+          tmem_ld_wait();
+          reg_fence(v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 p = ld_shared_cluster_f4(remote + (c * 32 + 4 * i) * 4);
+            const float s4[4] = {__uint_as_float(v[4 * i]) + p.x,
+                                 __uint_as_float(v[4 * i + 1]) + p.y,
+                                 __uint_as_float(v[4 * i + 2]) + p.z,
+                                 __uint_as_float(v[4 * i + 3]) + p.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int m = c * 32 + 4 * i + e;
+              if (m < M) C[size_t(m) * size_t(N) + n] = __float2bfloat16_rn(s4[e]);
+            }
+          }
+        }
+        mbar_arrive_cluster(mapa_shared(smem_u32(&part_done), 1));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+template <int NM, int STAGES>
+cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M, int N, int K,
+                           unsigned long long wait_limit_ns, unsigned int* err_word,
+                           cudaStream_t stream) {
+  using Cfg = SmallCfg<NM, STAGES>;
+  CUtensorMap tmA, tmW;
+  const uint64_t a_dims[2] = {uint64_t(K), uint64_t(M)};
+  const uint64_t w_dims[2] = {uint64_t(K), uint64_t(N)};
+  const uint64_t strides[1] = {uint64_t(K) * 2};
+  const uint32_t a_box[2] = {kBK, uint32_t(NM)};  // rows >= M read as zero
+  const uint32_t w_box[2] = {kBK, kSmallWRows};
+  if (!encode_tmap_bf16(&tmA, A, 2, a_dims, strides, a_box, true) ||
+      !encode_tmap_bf16(&tmW, W, 2, w_dims, strides, w_box, true))
+    return cudaErrorInvalidValue;
+  auto kern = oproj_small_m_kernel<NM, STAGES>;
+  static unsigned attr_done = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
+                                   &attr_done);
+  if (e != cudaSuccess) return e;
+  const int grid = (N / kSmallWRows) * 2;  // two CTAs (the K halves) per cluster
+  kern<<<grid, kSmallThreads, Cfg::kSmemBytes, stream>>>(tmA, tmW, C, M, N, K, wait_limit_ns,
+                                                        err_word);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int oproj_pick_bn(int64_t M, int N, int num_sms) {
@@ -268,11 +500,11 @@ int oproj_pick_bn(int64_t M, int N, int num_sms) {
   // times a per-tile efficiency of the narrower MMAs (measured on B200: an
   // M128 N64 MMA runs at ~0.7 of the N128/N256 rate per FLOP).
   const int64_t m_tiles = (M + kBM - 1) / kBM;
-  const int cand[4] = {256, 224, 128, 64};
-  const double tile_eff[4] = {1.0, 0.985, 0.95, 0.7};
-  int best = 64;
+  const int cand[3] = {256, 224, 128};
+  const double tile_eff[3] = {1.0, 0.985, 0.95};
+  int best = 128;
   double best_score = -1.0;
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 3; ++i) {
     const int bn = cand[i];
     if (N % bn != 0) continue;
     const int64_t tiles = m_tiles * (N / bn);
@@ -289,16 +521,21 @@ int oproj_pick_bn(int64_t M, int N, int num_sms) {
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
                               unsigned int* err_word, cudaStream_t stream) {
-  if (M <= 0 || N % 64 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
+  if (M <= 0 || N % 128 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
     return cudaErrorInvalidValue;
   CUtensorMap tmA;
   const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
   const uint64_t strides[1] = {uint64_t(K) * 2};
   const uint32_t box[2] = {kBK, kBM};
   if (!encode_tmap_bf16(&tmA, A, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
+  auto* Cb = static_cast<__nv_bfloat16*>(C);
+  if (!force_bn && M <= kSmallMMax && N % kSmallWRows == 0 && K % (2 * kBK) == 0) {
+    if (M <= 32) return launch_small_m<32, 9>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    if (M <= 64) return launch_small_m<64, 8>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    return launch_small_m<128, 6>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+  }
   const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
   if (N % bn != 0) return cudaErrorInvalidValue;
-  auto* Cb = static_cast<__nv_bfloat16*>(C);
   switch (bn) {
     case 256:
       return launch_bn<256, 4>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
@@ -308,9 +545,6 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
                                  stream);
     case 128:
       return launch_bn<128, 6>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
-                                 stream);
-    case 64:
-      return launch_bn<64, 8>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
                                  stream);
     default:
       return cudaErrorInvalidValue;

@@ -7,8 +7,10 @@
 namespace mla {
 
 // C[M, N] = A[M, K] . W[N, K]^T, all bf16 row-major, fp32 accumulation.
-// Requires N % 64 == 0, K % 64 == 0, 16-byte aligned pointers; the tile width
-// BN (64, 128, 224 or 256, dividing N) is chosen for wave efficiency unless
+// Requires N % 128 == 0, K % 64 == 0, 16-byte aligned pointers. M <= 128 (with
+// K % 128 == 0) runs the small-M kernel, which reads W once with two CTAs per
+// 128 rows of W (K halves) and swaps the MMA operands; otherwise the tile
+// width BN (128, 224 or 256, dividing N) is chosen for wave efficiency unless
 // `force_bn` (non-zero) fixes it.
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,

@@ -41,9 +41,11 @@ def check_status():
 
 
 # ------------------------------------------------------------------ o_proj
-@pytest.mark.parametrize("M", [1, 64, 129, 300, 1000])
+@pytest.mark.parametrize("M", [1, 31, 32, 33, 64, 100, 128, 129, 300, 1000])
 def test_oproj_all_rows(cuda_device, M):
-    """mla_o_proj on every row; M picks 64-, 128- and 256-wide tiles."""
+    """mla_o_proj on every row. M <= 128 runs the small-M kernel (token tile
+    of 32, 64 or 128, K split over a two-CTA cluster); larger M the tiled
+    GEMM with 128-, 224- or 256-wide tiles."""
     g = torch.Generator().manual_seed(M)
     attn = torch.randn(M, inputs.K_OPROJ, generator=g).to(torch.bfloat16)
     W = (torch.randn(inputs.D_MODEL, inputs.K_OPROJ, generator=g) * 0.02).to(torch.bfloat16)
