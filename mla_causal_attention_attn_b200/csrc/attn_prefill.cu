@@ -571,13 +571,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
       sc.kvalid = args.T - k0;
       sc.mask_vec = args.mask_vec;
-      // Causal kernel: keys c <= lim of the tile are allowed (c <= r on the
-      // query tile's own key tile, and none at or past the sequence's key
-      // count). `diag` marks the tiles where that limit cuts (warp-uniform).
-      const bool diag = !kMasked && (kt == qt || n_keys - k0 < kBKV);
-      const int lim = min(kt == qt ? r : kBKV - 1, n_keys - 1 - k0);
-      sc.diag_row = diag ? lim : kBKV;
-      const bool causal_fast = !kMasked && args.scale_log2 > 0.f;
+      // Keys c <= lim of the tile are allowed on the fast route below. Causal
+      // kernel: c <= r on the query tile's own key tile, and none at or past
+      // the sequence's key count. Masked kernel (fast route only on tiles
+      // whose mask entries are all zero): none at or past T. `diag` marks the
+      // tiles where that limit cuts (warp-uniform).
+      const bool diag = kMasked ? (args.T - k0 < kBKV) : (kt == qt || n_keys - k0 < kBKV);
+      const int lim = kMasked ? min(kBKV - 1, args.T - 1 - k0)
+                              : min(kt == qt ? r : kBKV - 1, n_keys - 1 - k0);
+      sc.diag_row = (!kMasked && diag) ? lim : kBKV;
+      // The fast route (scores need no mask add): every tile of the causal
+      // kernel, and the all-zero tiles of an explicit mask. It needs a
+      // positive scale (the raw maximum is then the scaled one).
+      const uint8_t tile_cls =
+          kMasked ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed)) : uint8_t(kTileZero);
+      const bool fast_route = tile_cls == kTileZero && args.scale_log2 > 0.f;
       uint32_t raw[kBKV];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -586,15 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence(raw);
       float alpha = 1.f;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
-      // Causal tiles after the first: one pass against the running max m,
+      // Fast-route tiles after the first: one pass against the running max m,
       // writing P (64 keys per store). Every p is then <= 2^8 unless the max
       // grew by more than the headroom, so a row sum <= 2^8 proves no rescale
       // is due; otherwise (rare: many keys near the max, or a new max) the
       // tile's true max is taken and, only if it grew past the headroom, the
       // tile is redone exactly below (new max, O rescaled). The first tile and
-      // the masked kernel always take the exact two-pass route. The choice is
-      // warp-uniform (a row whose max is still -inf fails the row-sum test).
-      bool exact = !(causal_fast && n > 0);
+      // the tiles that need their mask entries added take the exact two-pass
+      // route. The choice is warp-uniform (a row whose max is still -inf fails
+      // the row-sum test).
+      bool exact = !(fast_route && n > 0);
       float rowsum = 0.f;
       if (!exact) {
 #pragma unroll
@@ -625,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (exact) {
       float mt;
-      if (causal_fast) {
+      if (fast_route) {
         // positive scale: the maximum of the raw scores gives the maximum of
         // the scaled ones
         mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
@@ -662,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         const uint32_t* rc = raw + c * 32;
         uint32_t pk[16];
-        if (causal_fast) {
+        if (fast_route) {
           if (diag)
             p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
           else
