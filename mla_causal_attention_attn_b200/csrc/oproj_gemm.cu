@@ -530,9 +530,11 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
   if (!encode_tmap_bf16(&tmA, A, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
   auto* Cb = static_cast<__nv_bfloat16*>(C);
   if (!force_bn && M <= kSmallMMax && N % kSmallWRows == 0 && K % (2 * kBK) == 0) {
-    if (M <= 32) return launch_small_m<32, 9>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
-    if (M <= 64) return launch_small_m<64, 8>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
-    return launch_small_m<128, 6>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    // As many stages as shared memory holds: the kernel is bound by the bytes
+    // of W in flight.
+    if (M <= 32) return launch_small_m<32, 11>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    if (M <= 64) return launch_small_m<64, 9>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    return launch_small_m<128, 7>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
   }
   const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
   if (N % bn != 0) return cudaErrorInvalidValue;
