@@ -29,6 +29,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -104,9 +105,15 @@ def load_peaks():
 
 
 def kernel_source_sha(name):
+    """sha256[:16] of a kernel source's code: comments, trailing blanks and
+    blank lines removed, so that editing a comment keeps its ncu record."""
     p = os.path.join(ROOT, "mla_causal_attention_attn_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(p) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel_file, workload):

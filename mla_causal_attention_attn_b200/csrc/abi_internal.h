@@ -23,7 +23,8 @@ unsigned int* device_error_word();
 // Per-wait limit of the kernels' bounded waits (MLA_WAIT_LIMIT_NS, else 1 s).
 unsigned long long wait_limit_ns();
 
-// 1 when MLA_TEST_STALL_WAIT=1 (failure-detection tests only), else 0.
+// MLA_TEST_STALL_WAIT (failure-detection tests only): 1 stalls the attention
+// kernel, 2 the small-M o_proj; 0 when unset.
 int test_stall_wait();
 
 bool aligned16(const void* p);

@@ -17,22 +17,28 @@
 // every K/V tile brought into shared memory serves 256 query rows and the
 // softmax of one query tile overlaps the tensor-core work of the other.
 // Roles (384 threads = three warpgroups):
-//   warp 0       TMA producer: both Q tiles (nope + rope, 48 KB each) once,
-//                then for every visited 128-key tile five 16 KB blocks
-//                (k_nope lo/hi, the shared k_pe, v lo/hi) into an 8-block ring;
-//   warp 1       tensor-memory owner and MMA issuer. Per key tile j, in order:
-//                  O0 += P0_{j-1} V_{j-1},  S0 = Q0 K_j^T,
-//                  O1 += P1_{j-1} V_{j-1},  S1 = Q1 K_j^T
+//   warp 0       TMA producer: query tile 0 (nope + rope, 48 KB), the first key
+//                tile's K blocks, query tile 1, then for every visited 128-key
+//                tile five 16 KB blocks (k_nope lo/hi, the shared k_pe,
+//                v lo/hi) into an 8-block ring;
+//   warp 1       tensor-memory owner; warps 1 and 2: one MMA-issuing thread
+//                per query tile i, per key tile j in order
+//                  Oi += Pi_{j-1} V_{j-1},  Si = Qi K_j^T
 //                (S: 128x128, K = 128 nope + 64 rope, both operands in shared
-//                memory; PV: 128x128, K = 128 keys, P read from tensor memory).
-//                Because PV_{j-1} of a tile is issued before its S_j, the
-//                commit that announces S_j also guarantees O holds PV_{j-1};
-//   warps 2, 3   idle;
+//                memory; PV: 128x128, K = 128 keys, P read from tensor memory),
+//                with the S MMAs of the two tiles kept in the order
+//                S0_j, S1_j, S0_{j+1}, ... Because PV_{j-1} of a tile is issued
+//                before its S_j, the commit that announces S_j also guarantees
+//                O holds PV_{j-1};
+//   warp 3       idle;
 //   warps 4..7   softmax of query tile 0, one thread per row (TMEM lane);
 //   warps 8..11  softmax of query tile 1. Each reads S, scales, masks, keeps a
 //                running max (rescaling O only when the max grows by more than
 //                2^8), exponentiates, sums, writes P as bf16 over the first 64
 //                columns of its S buffer, and at the end O / l -> bf16 -> out.
+//                Tiles that need no mask entries added (every causal tile, the
+//                all-zero tiles of an explicit mask) take a single pass
+//                against the running max; the others two passes.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 #include "attn_prefill.h"
 #include "host_util.h"

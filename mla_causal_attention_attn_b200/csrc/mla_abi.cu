@@ -49,14 +49,16 @@ unsigned long long wait_limit_ns() {
   return v;
 }
 
-// MLA_TEST_STALL_WAIT=1 (read once) makes the attention kernel's first CTA
-// wait on a barrier that nothing completes, so that tests can check that the
-// bounded wait gives up, the CTA aborts cleanly and MLA_ERR_TIMEOUT is
-// reported. Never set in normal use.
+// MLA_TEST_STALL_WAIT (read once) lets tests make one bounded wait run out,
+// to check that the kernel gives up cleanly and MLA_ERR_TIMEOUT is reported:
+// 1 = the attention kernel's first CTA waits on a barrier that nothing
+// completes; 2 = in the first cluster of the small-M o_proj, the rank-1 CTA
+// never reports its partial sum. Never set in normal use.
 int test_stall_wait() {
   static const int v = [] {
     const char* s = std::getenv("MLA_TEST_STALL_WAIT");
-    return (s && s[0] == '1' && s[1] == '\0') ? 1 : 0;
+    if (s && (s[0] == '1' || s[0] == '2') && s[1] == '\0') return s[0] - '0';
+    return 0;
   }();
   return v;
 }
@@ -99,8 +101,8 @@ mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_n
   }
   return from_cuda(launch_attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld,
                                        mask ? cls : nullptr, B, T, softmax_scale, out,
-                                       wait_limit_ns(), device_error_word(), test_stall_wait(),
-                                       stream, valid_len));
+                                       wait_limit_ns(), device_error_word(),
+                                       test_stall_wait() == 1 ? 1 : 0, stream, valid_len));
 }
 
 }  // namespace abi
@@ -143,7 +145,8 @@ mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, ml
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_gemm(attn, W_o, out, M, MLA_HIDDEN, MLA_OPROJ_IN,
                                      device_sm_count(), wait_limit_ns(), 0, device_error_word(),
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     reinterpret_cast<cudaStream_t>(stream),
+                                     test_stall_wait() == 2 ? 1 : 0));
 }
 
 size_t mla_attn_oproj_workspace_bytes(int B, int T, int has_mask) {

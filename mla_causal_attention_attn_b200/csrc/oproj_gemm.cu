@@ -5,7 +5,7 @@
 //
 // Design (sm_100a):
 //   * persistent CTAs, one per SM, walking 128 x BN output tiles in a
-//     GROUP_M-swizzled order so concurrently running CTAs share A and W tiles
+//     row-block-grouped order so concurrently running CTAs share A and W tiles
 //     in L2;
 //   * warp 0 issues TMA loads of 128x64 A and BNx64 W tiles (128-byte
 //     swizzle) into a STAGES-deep shared-memory ring;
@@ -299,7 +299,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
     oproj_small_m_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmW, __nv_bfloat16* __restrict__ C,
                          int M, int N, int K, unsigned long long wait_limit_ns,
-                         unsigned int* err_word) {
+                         unsigned int* err_word, int test_stall) {
   using Cfg = SmallCfg<NM, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[STAGES];
@@ -429,7 +429,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
             dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                  __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
         }
-        mbar_arrive_cluster(mapa_shared(smem_u32(&part_ready), 0));
+        // (Failure-detection test: the first cluster's rank 1 never reports,
+        // so both CTAs' waits below must run out.)
+        if (!(test_stall && blockIdx.x == 1))
+          mbar_arrive_cluster(mapa_shared(smem_u32(&part_ready), 0));
         // Keep this CTA's shared memory until rank 0 has read the partial.
         mbar_wait_cluster(&part_done, 0, ctl, 8);
       } else if (mbar_wait_cluster(&part_ready, 0, ctl, 7)) {
@@ -471,7 +474,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
 template <int NM, int STAGES>
 cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M, int N, int K,
                            unsigned long long wait_limit_ns, unsigned int* err_word,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, int test_stall) {
   using Cfg = SmallCfg<NM, STAGES>;
   CUtensorMap tmA, tmW;
   const uint64_t a_dims[2] = {uint64_t(K), uint64_t(M)};
@@ -489,7 +492,7 @@ cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M
   if (e != cudaSuccess) return e;
   const int grid = (N / kSmallWRows) * 2;  // two CTAs (the K halves) per cluster
   kern<<<grid, kSmallThreads, Cfg::kSmemBytes, stream>>>(tmA, tmW, C, M, N, K, wait_limit_ns,
-                                                        err_word);
+                                                        err_word, test_stall);
   return cudaGetLastError();
 }
 
@@ -520,7 +523,7 @@ int oproj_pick_bn(int64_t M, int N, int num_sms) {
 
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
-                              unsigned int* err_word, cudaStream_t stream) {
+                              unsigned int* err_word, cudaStream_t stream, int test_stall) {
   if (M <= 0 || N % 128 != 0 || K % kBK != 0 || M > (int64_t(1) << 31) - kBM)
     return cudaErrorInvalidValue;
   CUtensorMap tmA;
@@ -532,9 +535,14 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
   if (!force_bn && M <= kSmallMMax && N % kSmallWRows == 0 && K % (2 * kBK) == 0) {
     // As many stages as shared memory holds: the kernel is bound by the bytes
     // of W in flight.
-    if (M <= 32) return launch_small_m<32, 11>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
-    if (M <= 64) return launch_small_m<64, 9>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
-    return launch_small_m<128, 7>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream);
+    if (M <= 32)
+      return launch_small_m<32, 11>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream,
+                                    test_stall);
+    if (M <= 64)
+      return launch_small_m<64, 9>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream,
+                                   test_stall);
+    return launch_small_m<128, 7>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream,
+                                  test_stall);
   }
   const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
   if (N % bn != 0) return cudaErrorInvalidValue;

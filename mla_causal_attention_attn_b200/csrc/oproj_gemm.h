@@ -12,9 +12,11 @@ namespace mla {
 // 128 rows of W (K halves) and swaps the MMA operands; otherwise the tile
 // width BN (128, 224 or 256, dividing N) is chosen for wave efficiency unless
 // `force_bn` (non-zero) fixes it.
+// test_stall (failure-detection tests only): in the first cluster of the
+// small-M kernel the rank-1 CTA never reports its partial sum.
 cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, int N, int K,
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
-                              unsigned int* err_word, cudaStream_t stream);
+                              unsigned int* err_word, cudaStream_t stream, int test_stall = 0);
 
 // Tile width the launcher picks for an M x N problem on `num_sms` SMs.
 int oproj_pick_bn(int64_t M, int N, int num_sms);
