@@ -45,13 +45,20 @@ __device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_ti
   nb = in_group / gm;
 }
 
-template <int BN, int STAGES>
+// An output tile is MT x 128 rows by BN columns. MT = 1: two accumulators in
+// tensor memory, so the epilogue of one tile overlaps the next tile's MMAs.
+// MT = 2: the two 128-row halves share each W tile (a third less L2 traffic
+// per FLOP) and fill the same columns, so there is one accumulator set.
+template <int BN, int STAGES, int MT>
 struct GemmCfg {
-  static constexpr uint32_t kABytes = kBM * kBK * 2;
+  static constexpr uint32_t kASub = kBM * kBK * 2;
+  static constexpr uint32_t kABytes = MT * kASub;
   static constexpr uint32_t kBBytes = BN * kBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  // two accumulators, rounded up to the power-of-two allocation granule
+  static constexpr int kNumAcc = MT == 1 ? 2 : 1;
+  // rounded up to the power-of-two allocation granule
   static constexpr uint32_t kTmemCols = 2 * BN <= 128 ? 128u : (2 * BN <= 256 ? 256u : 512u);
+  static_assert(MT == 1 || MT == 2, "MT");
   static constexpr size_t kSmemBytes = size_t(STAGES) * kStageBytes + 1024;
   static_assert(BN == 128 || BN == 224 || BN == 256, "BN");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -59,13 +66,13 @@ struct GemmCfg {
                 "TMEM columns must be a power of two in [32, 512]");
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     oproj_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, __nv_bfloat16* __restrict__ C,
                       int M, int N, int K, unsigned long long wait_limit_ns,
                       unsigned int* err_word) {
-  using Cfg = GemmCfg<BN, STAGES>;
+  using Cfg = GemmCfg<BN, STAGES, MT>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[STAGES];
   __shared__ uint64_t empty_bar[STAGES];
@@ -81,10 +88,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tiles = (M + kBM - 1) / kBM;
+  constexpr int kTileM = MT * kBM;
+  const int m_tiles = (M + kTileM - 1) / kTileM;
   const int n_tiles = N / BN;
   const int num_tiles = m_tiles * n_tiles;
   const int k_blocks = K / kBK;
+  // accumulator buffer of the local-th tile, and the parity of its use
+  auto acc_buf = [](int local) { return Cfg::kNumAcc == 2 ? (local & 1) : 0; };
+  auto acc_phase = [](int local) -> uint32_t {
+    return Cfg::kNumAcc == 2 ? uint32_t((local >> 1) & 1) : uint32_t(local & 1);
+  };
+  // TMEM column of the accumulator of row half t in buffer buf
+  auto acc_col = [](int buf, int t) -> uint32_t { return uint32_t((MT == 1 ? buf : t) * BN); };
 
   WaitCtl ctl{&abort_flag, wait_limit_ns, kErrKernelOproj, err_word};
 
@@ -130,7 +145,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sa = smem + size_t(stage) * Cfg::kStageBytes;
           uint8_t* sb = sa + Cfg::kABytes;
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
-          tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBK, mb * kBM);
+#pragma unroll
+          for (int t = 0; t < MT; ++t)
+            tma_load_2d(sa + t * Cfg::kASub, &tmA, &full_bar[stage], kb * kBK, mb * kTileM + t * kBM);
           tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBK, nb * BN);
           issued_mask |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -158,14 +175,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool issued_any = false;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
-        const int buf = local & 1;
-        const uint32_t acc_par = (local >> 1) & 1;
+        const int buf = acc_buf(local);
+        const uint32_t acc_par = acc_phase(local);
         if (!mbar_wait(&acc_empty[buf], acc_par ^ 1u, ctl, 3)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + uint32_t(buf * BN);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, ctl, 4)) {
             ok = false;
@@ -176,9 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = a_addr + Cfg::kABytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+              const uint64_t ad = sdesc_sw128(a_addr + t * Cfg::kASub + kk * 32, 16, 1024);
+              mma_ss(tmem_base + acc_col(buf, t), ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           issued_any = true;
           mma_commit(&empty_bar[stage]);  // frees the stage once these MMAs finish
@@ -205,16 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       int mb, nb;
       gemm_tile_coords(tile, m_tiles, n_tiles, mb, nb);
-      const int buf = local & 1;
-      const uint32_t acc_par = (local >> 1) & 1;
+      const int buf = acc_buf(local);
+      const uint32_t acc_par = acc_phase(local);
       if (!mbar_wait_warp(&acc_full[buf], acc_par, ctl, 6)) break;
       tc_fence_after();
-      const int row = mb * kBM + row_in_tile;
+#pragma unroll 1
+      for (int t = 0; t < MT; ++t) {
+      const int row = mb * kTileM + t * kBM + row_in_tile;
       __nv_bfloat16* crow = C + size_t(row) * size_t(N) + size_t(nb) * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem_addr(tmem_base, quad * 32, buf * BN + c * 32), r);
+        tmem_ld32(tmem_addr(tmem_base, quad * 32, acc_col(buf, t) + c * 32), r);
         tmem_ld_wait();
         reg_fence(r);
         uint32_t packed[16];
@@ -229,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 packed[4 * i + 3]);
         }
       }
+      }  // row halves
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
@@ -242,22 +264,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MT>
 cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, int M, int N,
                       int K, int num_sms, unsigned long long wait_limit_ns,
                       unsigned int* err_word, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN, STAGES>;
+  using Cfg = GemmCfg<BN, STAGES, MT>;
   CUtensorMap tmB;
   const uint64_t dims[2] = {uint64_t(K), uint64_t(N)};
   const uint64_t strides[1] = {uint64_t(K) * 2};
   const uint32_t box[2] = {kBK, BN};
   if (!encode_tmap_bf16(&tmB, W, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
-  auto kern = oproj_gemm_kernel<BN, STAGES>;
+  auto kern = oproj_gemm_kernel<BN, STAGES, MT>;
   static unsigned attr_done = 0;  // one bit per device ordinal
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
                                    &attr_done);
   if (e != cudaSuccess) return e;
-  const int m_tiles = (M + kBM - 1) / kBM;
+  const int m_tiles = (M + MT * kBM - 1) / (MT * kBM);
   const int num_tiles = m_tiles * (N / BN);
   const int grid = num_tiles < num_sms ? num_tiles : num_sms;
   kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(tmA, tmB, C, M, N, K, wait_limit_ns,
@@ -498,25 +520,25 @@ cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M
 
 }  // namespace
 
-int oproj_pick_bn(int64_t M, int N, int num_sms) {
+OprojTile oproj_pick_tile(int64_t M, int N, int num_sms) {
   // Largest expected throughput: fraction of the last wave's SMs kept busy,
-  // times a per-tile efficiency of the narrower tiles (measured on B200:
-  // 128x256 tiles ran 3 % faster than 128x224 at M = 16384, where both fill
-  // their last wave equally).
-  const int64_t m_tiles = (M + kBM - 1) / kBM;
-  const int cand[3] = {256, 224, 128};
-  const double tile_eff[3] = {1.0, 0.97, 0.95};
-  int best = 128;
+  // times a per-tile efficiency (measured on B200: 128x256 tiles ran 3 %
+  // faster than 128x224 at M = 16384, where both fill their last wave
+  // equally; 256x224 tiles ran 3-7 % faster than 128x224 at M = 16384 and
+  // 32768).
+  struct Cand { int bn, mt; double eff; };
+  const Cand cand[4] = {{256, 1, 1.0}, {224, 1, 0.97}, {128, 1, 0.95}, {224, 2, 1.03}};
+  OprojTile best{128, 1};
   double best_score = -1.0;
-  for (int i = 0; i < 3; ++i) {
-    const int bn = cand[i];
-    if (N % bn != 0) continue;
-    const int64_t tiles = m_tiles * (N / bn);
+  for (const Cand& c : cand) {
+    if (N % c.bn != 0) continue;
+    const int64_t m_tiles = (M + c.mt * kBM - 1) / (c.mt * kBM);
+    const int64_t tiles = m_tiles * (N / c.bn);
     const int64_t waves = (tiles + num_sms - 1) / num_sms;
-    const double score = double(tiles) / double(waves * num_sms) * tile_eff[i];
+    const double score = double(tiles) / double(waves * num_sms) * c.eff;
     if (score > best_score + 1e-9) {
       best_score = score;
-      best = bn;
+      best = OprojTile{c.bn, c.mt};
     }
   }
   return best;
@@ -545,17 +567,22 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
     return launch_small_m<128, 7>(A, W, Cb, int(M), N, K, wait_limit_ns, err_word, stream,
                                   test_stall);
   }
-  const int bn = force_bn ? force_bn : oproj_pick_bn(M, N, num_sms);
-  if (N % bn != 0) return cudaErrorInvalidValue;
-  switch (bn) {
+  const OprojTile tile = force_bn ? OprojTile{force_bn, 1} : oproj_pick_tile(M, N, num_sms);
+  if (N % tile.bn != 0) return cudaErrorInvalidValue;
+  if (tile.mt == 2) {
+    if (tile.bn != 224) return cudaErrorInvalidValue;
+    return launch_bn<224, 3, 2>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+                                stream);
+  }
+  switch (tile.bn) {
     case 256:
-      return launch_bn<256, 4>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+      return launch_bn<256, 4, 1>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
                                  stream);
     case 224:
-      return launch_bn<224, 5>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+      return launch_bn<224, 5, 1>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
                                  stream);
     case 128:
-      return launch_bn<128, 6>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
+      return launch_bn<128, 6, 1>(tmA, W, Cb, int(M), N, K, num_sms, wait_limit_ns, err_word,
                                  stream);
     default:
       return cudaErrorInvalidValue;

@@ -45,7 +45,7 @@ def check_status():
 def test_oproj_all_rows(cuda_device, M):
     """mla_o_proj on every row. M <= 128 runs the small-M kernel (token tile
     of 32, 64 or 128, K split over a two-CTA cluster); larger M the tiled
-    GEMM with 128-, 224- or 256-wide tiles."""
+    GEMM (M = 129: 128x128 tiles, 300: 128x224, 1000: 256x224)."""
     g = torch.Generator().manual_seed(M)
     attn = torch.randn(M, inputs.K_OPROJ, generator=g).to(torch.bfloat16)
     W = (torch.randn(inputs.D_MODEL, inputs.K_OPROJ, generator=g) * 0.02).to(torch.bfloat16)
@@ -56,8 +56,10 @@ def test_oproj_all_rows(cuda_device, M):
     assert_parity(to_f64(out), ref, f"o_proj M={M}")
 
 
-def test_oproj_large_sampled(cuda_device):
-    M = 4096 + 77
+@pytest.mark.parametrize("M", [4096 + 77, 8192 + 77])
+def test_oproj_large_sampled(cuda_device, M):
+    """Ragged large M, sampled rows: 256x224 tiles whose last tile has an empty
+    second row half (M = 4173), 128x256 tiles (M = 8269)."""
     g = torch.Generator().manual_seed(5)
     attn = torch.randn(M, inputs.K_OPROJ, generator=g).to(torch.bfloat16)
     W = (torch.randn(inputs.D_MODEL, inputs.K_OPROJ, generator=g) * 0.02).to(torch.bfloat16)
@@ -67,7 +69,7 @@ def test_oproj_large_sampled(cuda_device):
     rows = sorted(set([0, 1, 127, 128, 129, M - 1, M - 2, M - 78, M - 77]
                       + list(np.random.default_rng(0).integers(0, M, 100))))
     ref = oracle.oproj_rows(oracle.bf16_to_f64(attn[rows]), W)
-    assert_parity(to_f64(out[rows]), ref, "o_proj M=4173 sampled")
+    assert_parity(to_f64(out[rows]), ref, f"o_proj M={M} sampled")
 
 
 # ------------------------------------------------------------------ attention
