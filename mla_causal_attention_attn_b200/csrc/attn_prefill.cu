@@ -590,21 +590,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
       sc.kvalid = args.T - k0;
       sc.mask_vec = args.mask_vec;
-      // Keys c <= lim of the tile are allowed on the fast route below. Causal
-      // kernel: c <= r on the query tile's own key tile, and none at or past
-      // the sequence's key count. Masked kernel (fast route only on tiles
-      // whose mask entries are all zero): none at or past T. `diag` marks the
-      // tiles where that limit cuts (warp-uniform).
-      const bool diag = kMasked ? (args.T - k0 < kBKV) : (kt == qt || n_keys - k0 < kBKV);
-      const int lim = kMasked ? min(kBKV - 1, args.T - 1 - k0)
-                              : min(kt == qt ? r : kBKV - 1, n_keys - 1 - k0);
-      sc.diag_row = (!kMasked && diag) ? lim : kBKV;
       // The fast route (scores need no mask add): every tile of the causal
-      // kernel, and the all-zero tiles of an explicit mask. It needs a
-      // positive scale (the raw maximum is then the scaled one).
+      // kernel, and the all-zero and causal-pattern tiles of an explicit
+      // mask. It needs a positive scale (the raw maximum is then the scaled
+      // one).
       const uint8_t tile_cls =
           kMasked ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed)) : uint8_t(kTileZero);
-      const bool fast_route = tile_cls == kTileZero && args.scale_log2 > 0.f;
+      const bool causal_tile = !kMasked ? kt == qt : tile_cls == kTileCausal;
+      const bool fast_route =
+          (tile_cls == kTileZero || tile_cls == kTileCausal) && args.scale_log2 > 0.f;
+      // Keys c <= lim of the tile are allowed on the fast route: c <= r on a
+      // causal diagonal tile, and none at or past the sequence's key count
+      // (T, or valid_len[b]). `diag` marks the tiles where that limit cuts
+      // (warp-uniform).
+      const int key_end = kMasked ? args.T : n_keys;
+      const bool diag = causal_tile || key_end - k0 < kBKV;
+      const int lim = min(causal_tile ? r : kBKV - 1, key_end - 1 - k0);
+      sc.diag_row = (!kMasked && diag) ? lim : kBKV;
       uint32_t raw[kBKV];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -671,6 +673,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
             m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
           }
+          // keep the scaled, masked scores: the exponentials below need
+          // neither the mask nor the scale again
+#pragma unroll
+          for (int i = 0; i < 32; ++i) raw[c * 32 + i] = __float_as_uint(x[i]);
         }
         mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
@@ -697,7 +703,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
         } else {
           float x[32];
-          sc.apply(rc, c, args.scale_log2, m_use, x);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(rc[i]) - m_use;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float p0 = fast_exp2(x[2 * i]);
@@ -788,6 +795,10 @@ __global__ void __launch_bounds__(256)
   const uint16_t* base =
       reinterpret_cast<const uint16_t*>(mask) + (size_t(b) * T + q0) * mask_ld + k0;
   bool all_ninf = true, all_zero = true;
+  bool all_causal = kt == qt;  // diagonal tile: +-0 where key <= query, -inf above
+  auto causal_ok = [](uint32_t v, int rr, int c) {
+    return c <= rr ? (v & 0x7fffu) == 0u : v == 0xff80u;
+  };
   if (vec && cols == kBKV) {
     // 16 uint4 per row
     for (int idx = threadIdx.x; idx < rows * 16; idx += blockDim.x) {
@@ -799,6 +810,7 @@ __global__ void __launch_bounds__(256)
         const uint32_t lo = ws[e] & 0xffffu, hi = ws[e] >> 16;
         all_ninf &= (lo == 0xff80u) && (hi == 0xff80u);
         all_zero &= ((lo & 0x7fffu) == 0u) && ((hi & 0x7fffu) == 0u);
+        all_causal &= causal_ok(lo, rr, c8 * 8 + 2 * e) && causal_ok(hi, rr, c8 * 8 + 2 * e + 1);
       }
     }
   } else {
@@ -807,14 +819,17 @@ __global__ void __launch_bounds__(256)
       const uint32_t v = base[size_t(rr) * mask_ld + c];
       all_ninf &= (v == 0xff80u);
       all_zero &= ((v & 0x7fffu) == 0u);
+      all_causal &= causal_ok(v, rr, c);
     }
   }
   const int any_not_ninf = __syncthreads_or(!all_ninf);
   const int any_not_zero = __syncthreads_or(!all_zero);
+  const int any_not_causal = __syncthreads_or(!all_causal);
   if (threadIdx.x == 0) {
     uint8_t c = kTileMixed;
     if (!any_not_ninf) c = kTileSkip;
     else if (!any_not_zero) c = kTileZero;
+    else if (!any_not_causal) c = kTileCausal;
     cls[(size_t(b) * n_qt + qt) * n_kv + kt] = c;
   }
 }

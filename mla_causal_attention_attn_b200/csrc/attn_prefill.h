@@ -12,6 +12,8 @@ enum : uint8_t {
   kTileSkip = 0,   // every entry -inf: the tile contributes nothing
   kTileZero = 1,   // every entry +-0: scores need no mask add
   kTileMixed = 2,  // anything else: the kernel adds the mask entries
+  kTileCausal = 3, // a diagonal tile holding the causal pattern: +-0 where key <= query,
+                   // -inf above (no mask loads; the causal kernel's per-row limit)
 };
 
 // Bytes of the tile-class array for a [B,1,T,T] mask (B x ceil(T/128)^2).

@@ -129,6 +129,26 @@ def test_attn_general_additive_mask_and_fully_masked_rows(cuda_device):
     assert_parity(got[~rows_fm], ref[~rows_fm], "attn general mask")
 
 
+@pytest.mark.parametrize("B,T", [(1, 256), (2, 300)])
+def test_attn_explicit_causal_mask_is_the_causal_kernel(cuda_device, B, T):
+    """An explicit [B,1,T,T] causal mask (0 where key <= query, -inf above)
+    classifies into all-zero, causal-diagonal and skipped tiles, which take
+    the causal kernel's routes: the result is the causal call's, bit for bit."""
+    d = inputs.make_inputs(B, T, seed=31 + T, with_weight=False)
+    i = torch.arange(T).view(T, 1)
+    j = torch.arange(T).view(1, T)
+    m = torch.zeros(T, T)
+    m[j > i] = float("-inf")
+    d["mask"] = m.to(torch.bfloat16).expand(B, 1, T, T).contiguous()
+    g = to_dev(d, cuda_device)
+    explicit = gpu_attn(g)
+    g["mask"] = None
+    implicit = gpu_attn(g)
+    torch.cuda.synchronize()
+    check_status()
+    assert torch.equal(explicit, implicit)
+
+
 def test_attn_causal_future_invariance(cuda_device):
     """Rows <= t are bit-identical after changing keys/values at positions > t."""
     B, T, t = 1, 300, 140
