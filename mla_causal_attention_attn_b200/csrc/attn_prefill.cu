@@ -132,7 +132,8 @@ struct ScoreChunk {
   const __nv_bfloat16* mrow;  // mask row at the tile's first key (kMasked)
   int kvalid;                 // keys of the tile below T
   int mask_vec;               // 16-byte mask loads allowed
-  int diag_row;               // causal: keys c > diag_row are excluded
+  int diag_row;               // keys c > diag_row are excluded (the causal kernel's
+                              // diagonal; a causal-pattern or prefix tile of a mask)
 
   __device__ __forceinline__ void apply(const uint32_t* rr, int c, float scale_log2, float shift,
                                         float (&x)[32]) const {
@@ -150,6 +151,13 @@ struct ScoreChunk {
 #pragma unroll
       for (int i = 0; i < 32; ++i) x[i] = -INFINITY;
       return;
+    }
+    if (diag_row < kBKV) {
+      // causal-pattern and prefix tiles: their mask entries are +-0 up to the
+      // limit and -inf after it (only a non-positive scale brings them here)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c * 32 + i > diag_row) x[i] = -INFINITY;
     }
     if (cls == kTileMixed) {
       // 8 keys per 16-byte load when rows are 16-byte aligned; a chunk that
@@ -597,16 +605,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t tile_cls =
           kMasked ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed)) : uint8_t(kTileZero);
       const bool causal_tile = !kMasked ? kt == qt : tile_cls == kTileCausal;
+      const bool prefix_tile = kMasked && tile_cls >= kTilePrefix;
       const bool fast_route =
-          (tile_cls == kTileZero || tile_cls == kTileCausal) && args.scale_log2 > 0.f;
+          (tile_cls == kTileZero || tile_cls == kTileCausal || prefix_tile) &&
+          args.scale_log2 > 0.f;
       // Keys c <= lim of the tile are allowed on the fast route: c <= r on a
-      // causal diagonal tile, and none at or past the sequence's key count
-      // (T, or valid_len[b]). `diag` marks the tiles where that limit cuts
-      // (warp-uniform).
+      // causal diagonal tile, c <= the class's limit on a prefix tile, and
+      // none at or past the sequence's key count (T, or valid_len[b]). `diag`
+      // marks the tiles where that limit cuts (warp-uniform).
       const int key_end = kMasked ? args.T : n_keys;
-      const bool diag = causal_tile || key_end - k0 < kBKV;
-      const int lim = min(causal_tile ? r : kBKV - 1, key_end - 1 - k0);
-      sc.diag_row = (!kMasked && diag) ? lim : kBKV;
+      const bool diag = causal_tile || prefix_tile || key_end - k0 < kBKV;
+      const int lim = min(causal_tile ? r : (prefix_tile ? int(tile_cls) - kTilePrefix : kBKV - 1),
+                          key_end - 1 - k0);
+      sc.diag_row = (kMasked ? (causal_tile || prefix_tile) : diag) ? lim : kBKV;
       uint32_t raw[kBKV];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -782,9 +793,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- classifier
 // One pass over the additive mask: each 128x128 (query, key) tile, clipped to
-// T, becomes kTileSkip (every entry -inf), kTileZero (every entry +-0) or
-// kTileMixed. One CTA per tile, 256 threads, 16-byte loads when the rows are
-// 16-byte aligned (vec != 0), element loads otherwise.
+// T, becomes kTileSkip (every entry -inf), kTileZero (every entry +-0),
+// kTileCausal (the causal pattern on a diagonal tile), kTilePrefix + L (every
+// row +-0 on keys 0..L, -inf after) or kTileMixed. One CTA per tile, 256
+// threads, 16-byte loads when the rows are 16-byte aligned (vec != 0),
+// element loads otherwise.
 __global__ void __launch_bounds__(256)
     mask_tile_classify_kernel(const __nv_bfloat16* __restrict__ mask, int64_t mask_ld, int vec,
                               int T, int n_qt, int n_kv, uint8_t* __restrict__ cls) {
@@ -796,6 +809,20 @@ __global__ void __launch_bounds__(256)
       reinterpret_cast<const uint16_t*>(mask) + (size_t(b) * T + q0) * mask_ld + k0;
   bool all_ninf = true, all_zero = true;
   bool all_causal = kt == qt;  // diagonal tile: +-0 where key <= query, -inf above
+  // prefix pattern: every entry +-0 or -inf, the last +-0 column before the
+  // first -inf column in every row
+  bool zero_or_ninf = true;
+  int max_zero_col = -1, min_ninf_col = kBKV;
+  __shared__ int s_max_zero, s_min_ninf;
+  if (threadIdx.x == 0) {
+    s_max_zero = -1;
+    s_min_ninf = kBKV;
+  }
+  auto track = [&](uint32_t v, int c) {
+    if ((v & 0x7fffu) == 0u) max_zero_col = max(max_zero_col, c);
+    else if (v == 0xff80u) min_ninf_col = min(min_ninf_col, c);
+    else zero_or_ninf = false;
+  };
   auto causal_ok = [](uint32_t v, int rr, int c) {
     return c <= rr ? (v & 0x7fffu) == 0u : v == 0xff80u;
   };
@@ -811,6 +838,8 @@ __global__ void __launch_bounds__(256)
         all_ninf &= (lo == 0xff80u) && (hi == 0xff80u);
         all_zero &= ((lo & 0x7fffu) == 0u) && ((hi & 0x7fffu) == 0u);
         all_causal &= causal_ok(lo, rr, c8 * 8 + 2 * e) && causal_ok(hi, rr, c8 * 8 + 2 * e + 1);
+        track(lo, c8 * 8 + 2 * e);
+        track(hi, c8 * 8 + 2 * e + 1);
       }
     }
   } else {
@@ -820,16 +849,24 @@ __global__ void __launch_bounds__(256)
       all_ninf &= (v == 0xff80u);
       all_zero &= ((v & 0x7fffu) == 0u);
       all_causal &= causal_ok(v, rr, c);
+      track(v, c);
     }
   }
+  __syncthreads();  // s_max_zero / s_min_ninf initialised
+  atomicMax(&s_max_zero, max_zero_col);
+  atomicMin(&s_min_ninf, min_ninf_col);
   const int any_not_ninf = __syncthreads_or(!all_ninf);
   const int any_not_zero = __syncthreads_or(!all_zero);
   const int any_not_causal = __syncthreads_or(!all_causal);
+  const int any_other = __syncthreads_or(!zero_or_ninf);  // also orders the atomics
   if (threadIdx.x == 0) {
     uint8_t c = kTileMixed;
     if (!any_not_ninf) c = kTileSkip;
     else if (!any_not_zero) c = kTileZero;
     else if (!any_not_causal) c = kTileCausal;
+    else if (!any_other && s_max_zero >= 0 && s_max_zero + 1 == s_min_ninf &&
+             s_max_zero <= kBKV - 2)
+      c = uint8_t(kTilePrefix + s_max_zero);
     cls[(size_t(b) * n_qt + qt) * n_kv + kt] = c;
   }
 }

@@ -14,6 +14,8 @@ enum : uint8_t {
   kTileMixed = 2,  // anything else: the kernel adds the mask entries
   kTileCausal = 3, // a diagonal tile holding the causal pattern: +-0 where key <= query,
                    // -inf above (no mask loads; the causal kernel's per-row limit)
+  kTilePrefix = 4, // kTilePrefix + lim (lim in 0..126): every row is +-0 for the
+                   // tile's keys 0..lim and -inf after (no mask loads)
 };
 
 // Bytes of the tile-class array for a [B,1,T,T] mask (B x ceil(T/128)^2).

@@ -149,6 +149,83 @@ def test_attn_explicit_causal_mask_is_the_causal_kernel(cuda_device, B, T):
     assert torch.equal(explicit, implicit)
 
 
+def _prefix_mask(B, T, lens, causal):
+    """0 where key j < lens[b] (and j <= query i when causal), -inf elsewhere."""
+    i = torch.arange(T).view(T, 1)
+    j = torch.arange(T).view(1, T)
+    allowed = (j.unsqueeze(0) < torch.tensor(lens).view(-1, 1, 1)).expand(B, T, T)
+    if causal:
+        allowed = allowed & (j <= i).unsqueeze(0)
+    m = torch.full(allowed.shape, float("-inf"))
+    m.masked_fill_(allowed, 0.0)
+    return m.to(torch.bfloat16).unsqueeze(1).contiguous()
+
+
+def test_attn_prefix_mask_tiles_all_rows(cuda_device):
+    """A non-causal key-padding mask: every row of a tile allows the same key
+    prefix, so the tiles cut by the padding take the prefix route (above the
+    diagonal too; batch 3's in the ragged last key tile). Rows of batch 0 get
+    a staircase of per-row limits instead, which is no prefix and takes the
+    mixed route."""
+    B, T = 4, 300
+    d = inputs.make_inputs(B, T, seed=123, with_weight=False)
+    m = _prefix_mask(B, T, [300, 1, 150, 290], causal=False).float()
+    for i in range(T):
+        m[0, 0, i, 200 + i % 50:] = float("-inf")
+    d["mask"] = m.to(torch.bfloat16)
+    out = gpu_attn(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, fm = oracle_attn(d)
+    assert not fm.any()
+    assert_parity(to_f64(out).reshape(B * T, -1), ref, "attn prefix mask")
+
+
+def test_attn_keypad_dense_mask_matches_varlen(cuda_device):
+    """Causal attention with key padding, once as a dense mask and once as
+    valid_len: the dense form's all-zero, causal-diagonal and prefix tiles
+    take the same route as the compact form, so every row outside the query
+    tile holding the last valid key (whose diagonal tile is mixed in the
+    dense form) is the same, bit for bit."""
+    B, T, lens = 3, 700, [700, 333, 129]
+    d = inputs.make_inputs(B, T, seed=5, with_weight=False)
+    d["mask"] = _prefix_mask(B, T, lens, causal=True)
+    g = to_dev(d, cuda_device)
+    dense = gpu_attn(g)
+    compact = binding.attn_prefill_varlen(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                          torch.tensor(lens, dtype=torch.int32, device=cuda_device),
+                                          softmax_scale=g["softmax_scale"])
+    torch.cuda.synchronize()
+    check_status()
+    for b, L in enumerate(lens):
+        keep = torch.ones(T, dtype=torch.bool)
+        qt = (L - 1) // 128
+        if L < T:
+            keep[qt * 128:(qt + 1) * 128] = False
+        assert torch.equal(dense[b][keep], compact[b][keep]), f"b={b} L={L}"
+
+
+@pytest.mark.parametrize("scale_mul", [-1.0, 0.0])
+@pytest.mark.parametrize("form", ["causal", "causal_mask", "keypad_mask"])
+def test_attn_non_positive_scale(cuda_device, scale_mul, form):
+    """A negative or zero softmax scale takes the exact route on every tile,
+    where the causal cut, the causal-pattern tiles and the prefix tiles of a
+    mask are applied as explicit -inf entries."""
+    B, T = 2, 300
+    d = inputs.make_inputs(B, T, seed=41, with_weight=False)
+    d["softmax_scale"] = d["softmax_scale"] * scale_mul
+    if form == "causal_mask":
+        d["mask"] = _prefix_mask(B, T, [T, T], causal=True)
+    elif form == "keypad_mask":
+        d["mask"] = _prefix_mask(B, T, [170, 300], causal=True)
+    out = gpu_attn(to_dev(d, cuda_device))
+    torch.cuda.synchronize()
+    check_status()
+    ref, fm = oracle_attn(d)
+    assert not fm.any()
+    assert_parity(to_f64(out).reshape(B * T, -1), ref, f"attn scale*{scale_mul} {form}")
+
+
 def test_attn_causal_future_invariance(cuda_device):
     """Rows <= t are bit-identical after changing keys/values at positions > t."""
     B, T, t = 1, 300, 140
