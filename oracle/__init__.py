@@ -11,7 +11,10 @@ imports the other.
 
 What it follows: page "Kimi K2 · Mix and project", code excerpts
 modeling_deepseek.py 799-840 (query/key assembly, scaled scores, additive
-mask, fp32 softmax over keys, value mix) and 848-852 (head merge, o_proj).
+mask, fp32 softmax over keys, value mix) and 848-852 (head merge, o_proj);
+for the FP8 o_proj, page "Kimi K2 · Transformer blocks", configuration
+excerpt (quantization_config: e4m3 codes, dynamic activation scales,
+128 x 128 weight blocks), with the readings stated in mla_oracle.c.
 """
 from __future__ import annotations
 
@@ -60,6 +63,21 @@ def _load():
             lib.mla_oracle_oproj_rows.restype = ctypes.c_int
             lib.mla_oracle_oproj_rows.argtypes = [
                 f64p, u16p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, f64p]
+            f32p = ctypes.POINTER(ctypes.c_float)
+            lib.mla_oracle_e4m3_decode.restype = ctypes.c_double
+            lib.mla_oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.mla_oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.mla_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.mla_oracle_quant_rows_fp8.restype = ctypes.c_int
+            lib.mla_oracle_quant_rows_fp8.argtypes = [u16p, ctypes.c_int64, ctypes.c_int, u8p,
+                                                      f32p]
+            lib.mla_oracle_quant_weight_fp8.restype = ctypes.c_int
+            lib.mla_oracle_quant_weight_fp8.argtypes = [u16p, ctypes.c_int, ctypes.c_int, u8p,
+                                                        f32p]
+            lib.mla_oracle_oproj_fp8_rows.restype = ctypes.c_int
+            lib.mla_oracle_oproj_fp8_rows.argtypes = [
+                u8p, f32p, ctypes.c_int64, i64p, ctypes.c_int64, u8p, f32p, ctypes.c_int,
+                ctypes.c_int, f64p]
             lib.mla_oracle_num_threads.restype = ctypes.c_int
             lib.mla_oracle_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -177,3 +195,102 @@ def attn_oproj_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, W_o,
     attn, fm = attn_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale,
                          rows=rows)
     return oproj_rows(attn, W_o), fm.any(axis=1)
+
+
+# ------------------------------------------------------------------ FP8 o_proj
+# Page "Kimi K2 · Transformer blocks", configuration excerpt (config.json,
+# quantization_config: fp8, e4m3, dynamic activation scales, 128 x 128 weight
+# blocks). The arithmetic and the readings are in mla_oracle.c.
+
+FP8_GROUP = 128
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values (float64) of e4m3 codes (uint8 array-like)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    lib = _load()
+    flat = np.array([lib.mla_oracle_e4m3_decode(int(x)) for x in c.reshape(-1)],
+                    dtype=np.float64)
+    return flat.reshape(c.shape)
+
+
+def e4m3_encode(y) -> np.ndarray:
+    """Nearest e4m3 codes (ties to even, saturating at 448) of fp32 values."""
+    a = np.asarray(y, dtype=np.float32)
+    lib = _load()
+    flat = np.array([lib.mla_oracle_e4m3_encode(float(x)) for x in a.reshape(-1)],
+                    dtype=np.uint8)
+    return flat.reshape(a.shape)
+
+
+def quant_rows_fp8(x):
+    """Dynamic per-token quantisation of a bf16 [M, K] tensor.
+
+    Returns ``(q [M, K] uint8, scale [K/128, M] float32)``."""
+    bits = _bf16_bits(x)
+    if bits.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = bits.shape
+    q = np.zeros((M, K), dtype=np.uint8)
+    s = np.zeros((K // FP8_GROUP, M), dtype=np.float32)
+    rc = _load().mla_oracle_quant_rows_fp8(_ptr(bits, ctypes.c_uint16), ctypes.c_int64(M), K,
+                                           _ptr(q, ctypes.c_uint8), _ptr(s, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle quant_rows_fp8 failed ({rc})")
+    return q, s
+
+
+def quant_weight_fp8(W):
+    """128 x 128 block quantisation of a bf16 [N, K] weight.
+
+    Returns ``(q [N, K] uint8, scale [N/128, K/128] float32)``."""
+    bits = _bf16_bits(W)
+    if bits.ndim != 2:
+        raise ValueError("W must be [N, K]")
+    N, K = bits.shape
+    q = np.zeros((N, K), dtype=np.uint8)
+    s = np.zeros((N // FP8_GROUP, K // FP8_GROUP), dtype=np.float32)
+    rc = _load().mla_oracle_quant_weight_fp8(_ptr(bits, ctypes.c_uint16), N, K,
+                                             _ptr(q, ctypes.c_uint8), _ptr(s, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle quant_weight_fp8 failed ({rc})")
+    return q, s
+
+
+def _u8(a) -> np.ndarray:
+    import torch
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().contiguous().view(torch.uint8).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.uint8))
+
+
+def _f32(a) -> np.ndarray:
+    import torch
+    if isinstance(a, torch.Tensor):
+        a = a.detach().cpu().float().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def oproj_fp8_rows(qa, a_scale, qw, w_scale, rows=None) -> np.ndarray:
+    """Block-scaled e4m3 product for the requested rows of qa.
+
+    qa [M, K] codes, a_scale [K/128, M]; qw [N, K] codes, w_scale
+    [N/128, K/128]; rows: row indices or None for all. Returns [R, N] float64.
+    """
+    qa, qw = _u8(qa), _u8(qw)
+    a_scale, w_scale = _f32(a_scale), _f32(w_scale)
+    M, K = qa.shape
+    N = qw.shape[0]
+    if qw.shape[1] != K or a_scale.shape != (K // FP8_GROUP, M) or \
+            w_scale.shape != (N // FP8_GROUP, K // FP8_GROUP):
+        raise ValueError("fp8 operand shapes do not match")
+    r = (np.arange(M, dtype=np.int64) if rows is None
+         else np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1)))
+    out = np.zeros((r.shape[0], N), dtype=np.float64)
+    rc = _load().mla_oracle_oproj_fp8_rows(
+        _ptr(qa, ctypes.c_uint8), _ptr(a_scale, ctypes.c_float), ctypes.c_int64(M),
+        _ptr(r, ctypes.c_int64), ctypes.c_int64(r.shape[0]), _ptr(qw, ctypes.c_uint8),
+        _ptr(w_scale, ctypes.c_float), N, K, _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle oproj_fp8_rows failed ({rc})")
+    return out

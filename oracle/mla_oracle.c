@@ -17,6 +17,10 @@
  *     attn[b,i,h*Dv + e] = sum_j p_ij * v[b,h,j,e]
  *   out[r,n] = sum_k attn[r,k] * W_o[n,k]            (no bias)
  *
+ * and, for the FP8 form of o_proj (end of this file), the e4m3 codes, the
+ * dynamic per-token and 128 x 128 block quantisers and the block-scaled
+ * product.
+ *
  * - The query and key of every head are the concatenation of a non-rotary
  *   part and a rotary part; the key's rotary part is one tensor shared by all
  *   heads (the excerpt builds query_states / key_states that way, and the
@@ -230,6 +234,218 @@ int mla_oracle_oproj_rows(const double *a, const uint16_t *W, int64_t nrows,
         double acc = 0.0;
         for (int k = 0; k < K; ++k) acc += arow[k] * bf16_bits_to_double(wrow[k]);
         out[r * (int64_t)N + n] = acc;
+    }
+    return 0;
+}
+
+/* ================================================================ FP8 o_proj
+ *
+ * The checkpoint stores its projection weights as 8-bit floats (page "Kimi
+ * K2 · Transformer blocks", configuration excerpt moonshotai/Kimi-K2-Instruct
+ * config.json, quantization_config: quant_method fp8, fmt e4m3,
+ * activation_scheme dynamic, weight_block_size [128, 128]). The page gives
+ * those four fields and nothing more; the readings taken here:
+ *
+ * - e4m3 is the 8-bit float with 1 sign bit, 4 exponent bits (bias 7) and 3
+ *   mantissa bits: exponent field 0 holds the subnormals m * 2^-9, fields
+ *   1..15 hold (1 + m/8) * 2^(e-7), there are no infinities, and the two
+ *   codes with every exponent and mantissa bit set are NaN. The largest
+ *   finite value is 448.
+ * - weight_block_size [128, 128]: one fp32 scale per 128 x 128 block of
+ *   W_o [N, K], and W_o[n,k] ~= value(code[n,k]) * scale[n/128][k/128].
+ * - activation_scheme dynamic: the activations' scales are computed from the
+ *   data at run time, one per token and per 128-wide group of input
+ *   features (the weight block's extent along K).
+ * - A group's scale is amax / 448 in fp32 (1 for a group of zeros), and each
+ *   element's code is the e4m3 value nearest to x / scale, computed in fp32,
+ *   ties to the even code, magnitudes above 448 saturating to 448.
+ *
+ * The product is then, with a_s[g][m] the activation scales and w_s[j][g]
+ * the weight scales,
+ *   out[m,n] = sum_g a_s[g][m] * w_s[n/128][g]
+ *                    * sum_{k in group g} value(qa[m,k]) * value(qw[n,k]).
+ * Each group's inner sum is exact in double (the products of two e4m3
+ * values have at most 8 significant bits and span less than 2^40).
+ */
+
+#define FP8_GROUP 128
+#define E4M3_MAX 448.0
+
+/* Value of an e4m3 code, from the bit fields (NaN for the two NaN codes). */
+static double e4m3_value(uint8_t c)
+{
+    const int sign = c >> 7;
+    const int e = (c >> 3) & 15;
+    const int m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+double mla_oracle_e4m3_decode(uint8_t c) { return e4m3_value(c); }
+
+/*
+ * Code of the e4m3 value nearest to y: bisection over the non-negative finite
+ * codes 0..126 (their values increase with the code), ties to the code whose
+ * mantissa is even, |y| > 448 saturating to 448, the sign bit copied from y
+ * (so -0 and negatives that round to zero give 0x80).
+ */
+uint8_t mla_oracle_e4m3_encode(float y)
+{
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    if (isnan(y))
+        return (uint8_t)(sign | 0x7F);
+    const double a = fabs((double)y);
+    if (a >= E4M3_MAX)
+        return (uint8_t)(sign | 0x7E);
+    /* largest code lo with value(lo) <= a */
+    int lo = 0, hi = 126;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (e4m3_value((uint8_t)mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    uint8_t c = (uint8_t)lo;
+    if (lo < 126) {
+        const double below = a - e4m3_value((uint8_t)lo);
+        const double above = e4m3_value((uint8_t)(lo + 1)) - a;
+        if (above < below || (above == below && (lo & 1)))
+            c = (uint8_t)(lo + 1);
+    }
+    return (uint8_t)(sign | c);
+}
+
+/* Scale of a group whose largest magnitude is amax (fp32 arithmetic). */
+static float group_scale(float amax)
+{
+    return amax > 0.0f ? amax / 448.0f : 1.0f;
+}
+
+static float bf16_bits_to_float(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Codes of one group of n bf16 values at x (stride 1) with its scale. */
+static float quant_group(const uint16_t *x, int n, uint8_t *q)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        const float a = fabsf(bf16_bits_to_float(x[i]));
+        if (a > amax)
+            amax = a;
+    }
+    const float s = group_scale(amax);
+    for (int i = 0; i < n; ++i) {
+        const float y = bf16_bits_to_float(x[i]) / s;
+        q[i] = mla_oracle_e4m3_encode(y);
+    }
+    return s;
+}
+
+/*
+ * Dynamic activation quantisation: x [M, K] bf16 bits (row-major) ->
+ * q [M, K] e4m3 codes and scale [K/128][M] (group-major). Returns -1 on an
+ * argument error.
+ */
+int mla_oracle_quant_rows_fp8(const uint16_t *x, int64_t M, int K, uint8_t *q, float *scale)
+{
+    if (!x || !q || !scale || M < 1 || K < FP8_GROUP || K % FP8_GROUP != 0)
+        return -1;
+    const int G = K / FP8_GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int g = 0; g < G; ++g) {
+            const int64_t off = m * (int64_t)K + (int64_t)g * FP8_GROUP;
+            scale[(int64_t)g * M + m] = quant_group(x + off, FP8_GROUP, q + off);
+        }
+    return 0;
+}
+
+/*
+ * Block weight quantisation: W [N, K] bf16 bits -> q [N, K] e4m3 codes and
+ * scale [N/128][K/128]. Returns -1 on an argument error.
+ */
+int mla_oracle_quant_weight_fp8(const uint16_t *W, int N, int K, uint8_t *q, float *scale)
+{
+    if (!W || !q || !scale || N < FP8_GROUP || K < FP8_GROUP || N % FP8_GROUP != 0 ||
+        K % FP8_GROUP != 0)
+        return -1;
+    const int NB = N / FP8_GROUP, KB = K / FP8_GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t blk = 0; blk < (int64_t)NB * KB; ++blk) {
+        const int nb = (int)(blk / KB), kb = (int)(blk % KB);
+        float amax = 0.0f;
+        for (int r = 0; r < FP8_GROUP; ++r) {
+            const uint16_t *row = W + (int64_t)(nb * FP8_GROUP + r) * K + kb * FP8_GROUP;
+            for (int i = 0; i < FP8_GROUP; ++i) {
+                const float a = fabsf(bf16_bits_to_float(row[i]));
+                if (a > amax)
+                    amax = a;
+            }
+        }
+        const float s = group_scale(amax);
+        scale[blk] = s;
+        for (int r = 0; r < FP8_GROUP; ++r) {
+            const int64_t off = (int64_t)(nb * FP8_GROUP + r) * K + kb * FP8_GROUP;
+            for (int i = 0; i < FP8_GROUP; ++i)
+                q[off + i] = mla_oracle_e4m3_encode(bf16_bits_to_float(W[off + i]) / s);
+        }
+    }
+    return 0;
+}
+
+/*
+ * The block-scaled product for a list of rows:
+ *   out[r, n] = sum_g a_s[g][rows[r]] * w_s[n/128][g]
+ *                     * sum_{k in g} value(qa[rows[r], k]) * value(qw[n, k])
+ * qa [M, K] codes with a_scale [K/128][M]; qw [N, K] codes with
+ * w_scale [N/128][K/128]; out [nrows, N] double. Returns -1 on an argument
+ * error.
+ */
+int mla_oracle_oproj_fp8_rows(const uint8_t *qa, const float *a_scale, int64_t M,
+                              const int64_t *rows, int64_t nrows, const uint8_t *qw,
+                              const float *w_scale, int N, int K, double *out)
+{
+    if (!qa || !a_scale || !rows || !qw || !w_scale || !out || M < 1 || nrows < 0 ||
+        N < FP8_GROUP || K < FP8_GROUP || N % FP8_GROUP != 0 || K % FP8_GROUP != 0)
+        return -1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= M)
+            return -1;
+    double value[256];
+    for (int c = 0; c < 256; ++c)
+        value[c] = e4m3_value((uint8_t)c);
+    const int G = K / FP8_GROUP;
+    const int64_t work = nrows * (int64_t)N;
+#pragma omp parallel for schedule(static)
+    for (int64_t w = 0; w < work; ++w) {
+        const int64_t r = w / N;
+        const int n = (int)(w % N);
+        const int64_t m = rows[r];
+        const uint8_t *arow = qa + m * (int64_t)K;
+        const uint8_t *wrow = qw + (int64_t)n * K;
+        double acc = 0.0;
+        for (int g = 0; g < G; ++g) {
+            double block = 0.0;
+            for (int i = 0; i < FP8_GROUP; ++i) {
+                const int k = g * FP8_GROUP + i;
+                block += value[arow[k]] * value[wrow[k]];
+            }
+            acc += (double)a_scale[(int64_t)g * M + m] *
+                   (double)w_scale[(int64_t)(n / FP8_GROUP) * G + g] * block;
+        }
+        out[w] = acc;
     }
     return 0;
 }
