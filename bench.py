@@ -20,6 +20,11 @@ the max over ranks.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of rows of the
 same workload (rank 0 only), as the reference arm.
+
+--oproj fp8 runs o_proj in the checkpoint's FP8 form instead: W_o quantised
+once to e4m3 with 128 x 128 block scales before timing, and in every step the
+attention output quantised per token and 128-feature group, then the
+block-scaled e4m3 GEMM (the step's o_proj time covers both kernels).
 """
 from __future__ import annotations
 
@@ -47,6 +52,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 LONG_REGION_S = 0.5
 # o_proj of at most this many rows runs the HBM-bound small-M kernel.
 SMALL_M_MAX = 128
+# Dense e4m3 against bf16 tensor throughput (nominal 4.5 / 2.25 PFLOP/s).
+FP8_OVER_BF16 = 2.0
 
 
 # ---------------------------------------------------------------- FLOP counts
@@ -258,8 +265,8 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, flushed=True):
-    return {
+def workload_config(w, flushed=True, oproj="bf16"):
+    cfg = {
         "workload": w.name, "B": w.B, "T": w.T, "heads": H,
         "qk_head_dim": "128 nope + 64 rope (rope key shared by all heads)", "v_head_dim": DV,
         "o_proj": "8192 -> 7168",
@@ -270,6 +277,10 @@ def workload_config(w, flushed=True):
         if flushed else "n/a",
         "parallelism": "independent batch per GPU (no collective)",
     }
+    if oproj == "fp8":
+        cfg["o_proj"] = ("8192 -> 7168, e4m3 operands: W_o in 128x128 blocks (quantised before "
+                         "timing), activations per token and 128-feature group (in the step)")
+    return cfg
 
 
 def run_ours(args, w, rank, world, local_rank):
@@ -288,7 +299,12 @@ def run_ours(args, w, rank, world, local_rank):
     names = ["q_nope", "q_pe", "k_nope", "k_pe", "v"] + extra
     g = {k: d[k].to(dev) for k in names}
     W = d["W_o"].to(dev)
+    fp8 = args.oproj == "fp8"
     B, T = w.B, w.T
+    if fp8:
+        W_q, W_s = binding.quantize_weight_fp8(W)
+        a_q = torch.empty((B * T, K_OPROJ), dtype=torch.uint8, device=dev)
+        a_s = torch.empty((K_OPROJ // 128, B * T), dtype=torch.float32, device=dev)
     dense_mask = d["mask"] is not None and not compact
     ws_attn = torch.empty(binding.attn_prefill_workspace_bytes(B, T, dense_mask) or 16,
                           dtype=torch.uint8, device=dev)
@@ -311,7 +327,13 @@ def run_ours(args, w, rank, world, local_rank):
                                  workspace=ws_attn, stream=stream)
         if ev:
             ev[1].record(stream)
-        binding.o_proj(attn, W, out=out, stream=stream)
+        if fp8:
+            binding.quantize_act_fp8(attn, q=a_q, scale=a_s, stream=stream)
+            if ev:
+                ev[3].record(stream)
+            binding.o_proj_fp8(a_q, a_s, W_q, W_s, out=out.view(-1, D_MODEL), stream=stream)
+        else:
+            binding.o_proj(attn, W, out=out, stream=stream)
         if ev:
             ev[2].record(stream)
 
@@ -323,7 +345,8 @@ def run_ours(args, w, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 if fp8 else 3)]
+           for _ in range(args.steps)]
     sampler = ClockSampler(gpu_uuid(dev)) if rank == 0 else None
     if world > 1:
         dist.barrier()
@@ -346,6 +369,8 @@ def run_ours(args, w, rank, world, local_rank):
 
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     oproj_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    quant_ms = [e[1].elapsed_time(e[3]) for e in evs] if fp8 else None
+    gemm_ms = [e[3].elapsed_time(e[2]) for e in evs] if fp8 else oproj_ms
     step_ms = [a + b for a, b in zip(attn_ms, oproj_ms)]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
 
@@ -371,7 +396,8 @@ def run_ours(args, w, rank, world, local_rank):
         for i in range(2):
             sets.append({
                 "in": g if i == 0 else {k: torch.empty_like(g[k]) for k in names},
-                "ws": torch.empty(binding.attn_oproj_workspace_bytes(B, T, dense_mask),
+                "ws": torch.empty((binding.attn_oproj_fp8_workspace_bytes if fp8 else
+                                   binding.attn_oproj_workspace_bytes)(B, T, dense_mask),
                                   dtype=torch.uint8, device=dev),
                 "out": out if i == 0 else torch.empty_like(out),
                 "out_h": torch.empty((B, T, D_MODEL), dtype=torch.bfloat16).pin_memory(),
@@ -391,7 +417,12 @@ def run_ours(args, w, rank, world, local_rank):
             stream.wait_event(bs["in_done"])
             if k >= 2:
                 stream.wait_event(bs["out_done"])    # step k-2's output has left
-            if compact:
+            if fp8:
+                binding.attn_oproj_fp8(gi["q_nope"], gi["q_pe"], gi["k_nope"], gi["k_pe"],
+                                       gi["v"], W_q, W_s, mask=gi.get("mask"),
+                                       softmax_scale=scale, out=bs["out"], workspace=bs["ws"],
+                                       stream=stream)
+            elif compact:
                 binding.attn_oproj_varlen(gi["q_nope"], gi["q_pe"], gi["k_nope"], gi["k_pe"],
                                           gi["v"], gi["valid_len_i32"], W, softmax_scale=scale,
                                           out=bs["out"], workspace=bs["ws"], stream=stream)
@@ -422,7 +453,8 @@ def run_ours(args, w, rank, world, local_rank):
         e2e = {"value": job_tflops(world, flops_step, n_e2e, e2e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e2e_ms / n_e2e,
-               "call": "mla_attn_oproj_varlen" if compact else "mla_attn_oproj",
+               "call": ("mla_attn_oproj_fp8" if fp8 else
+                        "mla_attn_oproj_varlen" if compact else "mla_attn_oproj"),
                "note": "per step: pinned H2D of the activations (and mask or valid lengths), "
                        "the fused call, D2H of the output; steps overlap on copy-in / compute "
                        "/ copy-out streams with two device buffer sets; W_o resident like any "
@@ -433,9 +465,11 @@ def run_ours(args, w, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     a_avg = statistics.mean(attn_ms)
     o_avg = statistics.mean(oproj_ms)
-    small_m = B * T <= SMALL_M_MAX
+    g_avg = statistics.mean(gemm_ms)
+    small_m = B * T <= SMALL_M_MAX and not fp8
     kern = {"attn": (fa, a_avg, "attn_prefill.cu", "mla_attn_prefill_kernel"),
-            "oproj": (fo, o_avg, "oproj_gemm.cu",
+            "oproj": (fo, g_avg, "fp8_oproj.cu" if fp8 else "oproj_gemm.cu",
+                      "oproj_fp8_kernel" if fp8 else
                       "oproj_small_m_kernel" if small_m else "oproj_gemm_kernel")}
     dom = max(kern, key=lambda k: kern[k][1])
     f_dom, t_dom, src_dom, kname = kern[dom]
@@ -457,14 +491,18 @@ def run_ours(args, w, rank, world, local_rank):
         # the burst peak. Both fractions are reported.
         long_region = wall >= LONG_REGION_S
         peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        # An e4m3 contraction takes the bf16 peak times the nominal ratio.
+        mul = FP8_OVER_BF16 if (fp8 and dom == "oproj") else 1.0
         roofline = {"kernel": kname, "bound": "tensor", "achieved": achieved,
-                    "peak": peaks[peak_key], "unit": "TFLOP/s",
-                    "frac": achieved / peaks[peak_key],
+                    "peak": mul * peaks[peak_key], "unit": "TFLOP/s",
+                    "frac": achieved / (mul * peaks[peak_key]),
                     "peak_source": f"{peak_src} bf16 " + (
                         f"sustained (timed region {wall:.2f} s)" if long_region
-                        else f"burst (timed region {wall:.2f} s)"),
-                    "frac_of_burst": achieved / peaks["bf16_tflops"],
-                    "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                        else f"burst (timed region {wall:.2f} s)") + (
+                        f" x {FP8_OVER_BF16:g} (nominal e4m3 : bf16 dense ratio)"
+                        if mul != 1.0 else ""),
+                    "frac_of_burst": achieved / (mul * peaks["bf16_tflops"]),
+                    "frac_of_sustained": achieved / (mul * peaks["bf16_tflops_sustained"]),
                     "traffic": recorded_traffic(src_dom, w.name),
                     "per_launch_flops": f_dom, "avg_launch_ms": t_dom}
     cpu = None
@@ -473,20 +511,22 @@ def run_ours(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 attention, e4m3 o_proj" if fp8 else "bf16",
         "data": "synthetic (seeded: activations N(0,1), W_o N(0,0.02))",
-        "config": workload_config(w),
+        "config": workload_config(w, oproj=args.oproj),
         "pct_of_peak": {"measured_bf16_burst": 100 * value / peaks["bf16_tflops"],
                         "measured_bf16_sustained": 100 * value / peaks["bf16_tflops_sustained"],
                         "datasheet_dense_bf16": 100 * value / DATASHEET_BF16_TFLOPS,
                         "peak_source": peak_src},
-        "kernels_ms": {"attn": a_avg, "oproj": o_avg},
+        "kernels_ms": ({"attn": a_avg, "oproj": o_avg, "oproj_quant": statistics.mean(quant_ms),
+                        "oproj_gemm": g_avg} if fp8 else {"attn": a_avg, "oproj": o_avg}),
         "flops_per_step": {"attn": fa, "oproj": fo},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks,
-        "gpu_launches": args.steps * (2 + (1 if dense_mask else 0)),
+        "gpu_launches": args.steps * (2 + (1 if dense_mask else 0) + (1 if fp8 else 0)),
         "wall_s_timed_region": wall,
     }
     print(json.dumps(line), flush=True)
@@ -513,12 +553,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--oproj", choices=["bf16", "fp8"], default="bf16")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     from mla_causal_attention_attn_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
+    if args.oproj == "fp8" and (w.compact_mask or args.impl == "reference"):
+        ap.error("--oproj fp8 runs with the dense-mask or causal workloads of the ours arm")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 2
+#define MLA_ABI_VERSION 3
 
 /* Model dimensions (fixed at compile time; no other values are accepted). */
 #define MLA_NUM_HEADS 64
@@ -203,6 +203,84 @@ mla_status_t mla_attn_oproj_noalloc(const mla_bf16* q_nope, const mla_bf16* q_pe
                                     const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld,
                                     int B, int T, float softmax_scale, const mla_bf16* W_o,
                                     mla_bf16* out, mla_stream_t stream);
+
+/*
+ * ------------------------------------------------------------ FP8 o_proj
+ * The checkpoint stores o_proj as 8-bit floats (page "Kimi K2 · Transformer
+ * blocks", configuration excerpt config.json, quantization_config:
+ * quant_method fp8, fmt e4m3, activation_scheme dynamic, weight_block_size
+ * [128, 128]). The calls below use that format, read as follows:
+ *  - codes: e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ *    infinities, largest finite value 448), one byte per element;
+ *  - weights: one fp32 scale per 128 x 128 block, W_o ~= value(code) * scale;
+ *  - activations ("dynamic"): scales computed at run time, one per token and
+ *    per 128-wide group of the 8192 input features;
+ *  - a group's scale is amax / 448 in fp32 (1 for a group of zeros) and each
+ *    code is the e4m3 value nearest to x / scale computed in fp32, ties to
+ *    the even code, saturating at +-448;
+ *  - the product: out[m,n] = sum_g a_scale[g][m] * W_scale[n/128][g] *
+ *    sum over the group's 128 features of value(a) * value(W), accumulated in
+ *    fp32 and rounded once to bf16.
+ * Inputs must be finite.
+ */
+
+/* Quantisation groups along the 8192 input features, and weight blocks along
+ * the 7168 outputs. */
+#define MLA_FP8_GROUP 128
+#define MLA_FP8_K_GROUPS 64  /* MLA_OPROJ_IN / MLA_FP8_GROUP */
+#define MLA_FP8_N_BLOCKS 56  /* MLA_HIDDEN / MLA_FP8_GROUP */
+
+/*
+ * Dynamic activation quantisation:
+ *   x      [M, 8192] bf16 (row-major, contiguous)
+ *   M      rows, 1 .. 2^31 - 129
+ *   q      [M, 8192] e4m3 codes (uint8)
+ *   scale  [64, M] fp32, group-major: scale[g * M + m] for features
+ *          128g .. 128g+127 of row m
+ */
+mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, float* scale,
+                                  mla_stream_t stream);
+
+/*
+ * Block weight quantisation of W_o (done once, like loading a checkpoint):
+ *   W      [7168, 8192] bf16 (out_features, in_features)
+ *   q      [7168, 8192] e4m3 codes
+ *   scale  [56, 64] fp32: scale[nb * 64 + g] for rows 128nb.. and features 128g..
+ */
+mla_status_t mla_quantize_weight_fp8(const mla_bf16* W, uint8_t* q, float* scale,
+                                     mla_stream_t stream);
+
+/*
+ * o_proj on e4m3 operands (the product above):
+ *   attn_q      [M, 8192] codes, attn_scale [64, M] (from mla_quantize_act_fp8)
+ *   W_q         [7168, 8192] codes, W_scale [56, 64] (from mla_quantize_weight_fp8
+ *               or a checkpoint in that layout)
+ *   M           rows, 1 .. 2^31 - 129
+ *   out         [M, 7168] bf16
+ * Code pointers and out 16-byte aligned; scale pointers 4-byte aligned.
+ */
+mla_status_t mla_o_proj_fp8(const uint8_t* attn_q, const float* attn_scale, const uint8_t* W_q,
+                            const float* W_scale, int64_t M, mla_bf16* out, mla_stream_t stream);
+
+/*
+ * Workspace bytes mla_attn_oproj_fp8 needs: the merged bf16 attention output
+ * (B*T*8192*2), its codes (B*T*8192) and scales (64*B*T*4), each rounded up
+ * to 256, plus the mask-class bytes when has_mask != 0. Returns 0 for B < 1
+ * or T < 1.
+ */
+size_t mla_attn_oproj_fp8_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * mla_attn_oproj with an FP8 o_proj: attention, dynamic quantisation of its
+ * merged output, then mla_o_proj_fp8 with the quantised W_o. Arguments as in
+ * mla_attn_oproj, with W_q / W_scale in place of W_o.
+ */
+mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                                int T, float softmax_scale, const uint8_t* W_q,
+                                const float* W_scale, void* workspace, size_t workspace_bytes,
+                                mla_bf16* out, mla_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

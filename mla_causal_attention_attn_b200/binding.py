@@ -54,6 +54,14 @@ _SIGNATURES = {
     "mla_attn_oproj_varlen": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_float, _VP, _VP,
                                              ctypes.c_size_t, _VP, _VP]),
+    "mla_quantize_act_fp8": (ctypes.c_int, [_VP, ctypes.c_int64, _VP, _VP, _VP]),
+    "mla_quantize_weight_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP]),
+    "mla_o_proj_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]),
+    "mla_attn_oproj_fp8_workspace_bytes": (ctypes.c_size_t,
+                                           [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_oproj_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_float, _VP, _VP,
+                                          _VP, ctypes.c_size_t, _VP, _VP]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_abi_version": (ctypes.c_int, []),
@@ -288,6 +296,103 @@ def attn_oproj_noalloc(q_nope, q_pe, k_nope, k_pe, v, W_o, mask=None, softmax_sc
                                     _ptr(mask), mask_ld, B, T, scale, _ptr(W_o), _ptr(out),
                                     _stream_handle(stream))
     _check("mla_attn_oproj_noalloc", st)
+    return out
+
+
+# ------------------------------------------------------------------ FP8 o_proj
+FP8_GROUP = 128
+FP8_K_GROUPS = K_OPROJ // FP8_GROUP
+FP8_N_BLOCKS = D_MODEL // FP8_GROUP
+
+
+def _req_t(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def quantize_act_fp8(x, q=None, scale=None, stream=None):
+    """Dynamic e4m3 quantisation of ``x [M, 8192]`` (bf16) via
+    ``mla_quantize_act_fp8``: codes [M, 8192] (uint8), scales [64, M] (fp32)."""
+    lib = load()
+    x2 = x.reshape(-1, K_OPROJ)
+    M = x2.shape[0]
+    _req(x2, (M, K_OPROJ), "x")
+    if q is None:
+        q = torch.empty((M, K_OPROJ), dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((FP8_K_GROUPS, M), dtype=torch.float32, device=x.device)
+    _req_t(q, torch.uint8, (M, K_OPROJ), "q")
+    _req_t(scale, torch.float32, (FP8_K_GROUPS, M), "scale")
+    st = lib.mla_quantize_act_fp8(_ptr(x2), M, _ptr(q), _ptr(scale), _stream_handle(stream))
+    _check("mla_quantize_act_fp8", st)
+    return q, scale
+
+
+def quantize_weight_fp8(W_o, stream=None):
+    """128 x 128 block e4m3 quantisation of ``W_o [7168, 8192]`` via
+    ``mla_quantize_weight_fp8``: codes [7168, 8192], scales [56, 64]."""
+    lib = load()
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    q = torch.empty((D_MODEL, K_OPROJ), dtype=torch.uint8, device=W_o.device)
+    scale = torch.empty((FP8_N_BLOCKS, FP8_K_GROUPS), dtype=torch.float32, device=W_o.device)
+    st = lib.mla_quantize_weight_fp8(_ptr(W_o), _ptr(q), _ptr(scale), _stream_handle(stream))
+    _check("mla_quantize_weight_fp8", st)
+    return q, scale
+
+
+def o_proj_fp8(attn_q, attn_scale, W_q, W_scale, out=None, stream=None):
+    """Block-scaled e4m3 o_proj -> [M, 7168] bf16 via ``mla_o_proj_fp8``."""
+    lib = load()
+    M = attn_q.shape[0]
+    _req_t(attn_q, torch.uint8, (M, K_OPROJ), "attn_q")
+    _req_t(attn_scale, torch.float32, (FP8_K_GROUPS, M), "attn_scale")
+    _req_t(W_q, torch.uint8, (D_MODEL, K_OPROJ), "W_q")
+    _req_t(W_scale, torch.float32, (FP8_N_BLOCKS, FP8_K_GROUPS), "W_scale")
+    if out is None:
+        out = torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=attn_q.device)
+    _req(out.view(-1, D_MODEL), (M, D_MODEL), "out")
+    st = lib.mla_o_proj_fp8(_ptr(attn_q), _ptr(attn_scale), _ptr(W_q), _ptr(W_scale), M,
+                            _ptr(out), _stream_handle(stream))
+    _check("mla_o_proj_fp8", st)
+    return out
+
+
+def attn_oproj_fp8_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_oproj_fp8_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def attn_oproj_fp8(q_nope, q_pe, k_nope, k_pe, v, W_q, W_scale, mask=None, softmax_scale=None,
+                   out=None, workspace=None, stream=None):
+    """Attention, dynamic e4m3 quantisation of its output, FP8 o_proj:
+    [B, T, 7168] bf16 via ``mla_attn_oproj_fp8``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _req_t(W_q, torch.uint8, (D_MODEL, K_OPROJ), "W_q")
+    _req_t(W_scale, torch.float32, (FP8_N_BLOCKS, FP8_K_GROUPS), "W_scale")
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    need = attn_oproj_fp8_workspace_bytes(B, T, mask is not None)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.mla_attn_oproj_fp8(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                _ptr(mask), mask_ld, B, T, scale, _ptr(W_q), _ptr(W_scale),
+                                _ptr(workspace), ws_bytes, _ptr(out), _stream_handle(stream))
+    _check("mla_attn_oproj_fp8", st)
     return out
 
 

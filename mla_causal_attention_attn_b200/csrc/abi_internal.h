@@ -28,6 +28,7 @@ unsigned long long wait_limit_ns();
 int test_stall_wait();
 
 bool aligned16(const void* p);
+bool aligned4(const void* p);
 size_t round_up(size_t x, size_t a);
 
 // MLA_ERR_UNSUPPORTED_DEVICE unless the current device is CC 10.0.

@@ -16,6 +16,10 @@ namespace mla {
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                       const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
 
+// Same for a tensor of bytes (e4m3 codes): dims and box in elements = bytes.
+bool encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
 // Number of SMs of the current device (cached per device ordinal).
 int device_sm_count();
 

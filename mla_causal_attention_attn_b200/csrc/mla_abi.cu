@@ -7,6 +7,7 @@
 #include "../../include/mla.h"
 #include "abi_internal.h"
 #include "attn_prefill.h"
+#include "fp8_oproj.h"
 #include "host_util.h"
 #include "oproj_gemm.h"
 #include "sm100.cuh"
@@ -64,6 +65,8 @@ int test_stall_wait() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -224,6 +227,89 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
   return from_cuda(launch_oproj_gemm(workspace, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
                                      device_sm_count(), wait_limit_ns(), 0, device_error_word(),
                                      st));
+}
+
+mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, float* scale,
+                                  mla_stream_t stream) {
+  if (!x || !q || !scale) return MLA_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(q) || !aligned4(scale)) return MLA_ERR_MISALIGNED;
+  mla_status_t s = check_device();
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_quant_rows_fp8(x, MLA_OPROJ_IN, M, MLA_OPROJ_IN, q, scale,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mla_status_t mla_quantize_weight_fp8(const mla_bf16* W, uint8_t* q, float* scale,
+                                     mla_stream_t stream) {
+  if (!W || !q || !scale) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(q) || !aligned4(scale)) return MLA_ERR_MISALIGNED;
+  mla_status_t s = check_device();
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_quant_weight_fp8(W, MLA_HIDDEN, MLA_OPROJ_IN, q, scale,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mla_status_t mla_o_proj_fp8(const uint8_t* attn_q, const float* attn_scale, const uint8_t* W_q,
+                            const float* W_scale, int64_t M, mla_bf16* out,
+                            mla_stream_t stream) {
+  if (!attn_q || !attn_scale || !W_q || !W_scale || !out) return MLA_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
+  if (!aligned16(attn_q) || !aligned16(W_q) || !aligned16(out) || !aligned4(attn_scale) ||
+      !aligned4(W_scale))
+    return MLA_ERR_MISALIGNED;
+  mla_status_t s = check_device();
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_fp8(attn_q, attn_scale, W_q, W_scale, out, M, MLA_HIDDEN,
+                                    MLA_OPROJ_IN, device_sm_count(), wait_limit_ns(),
+                                    device_error_word(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_attn_oproj_fp8_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  const size_t M = size_t(B) * size_t(T);
+  size_t bytes = round_up(M * MLA_OPROJ_IN * 2, 256) + round_up(M * MLA_OPROJ_IN, 256) +
+                 round_up(M * MLA_FP8_K_GROUPS * 4, 256);
+  if (has_mask) bytes += round_up(attn_class_bytes(B, T), 256);
+  return bytes;
+}
+
+mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
+                                const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
+                                int T, float softmax_scale, const uint8_t* W_q,
+                                const float* W_scale, void* workspace, size_t workspace_bytes,
+                                mla_bf16* out, mla_stream_t stream) {
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if (!W_q || !W_scale) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_q) || !aligned4(W_scale)) return MLA_ERR_MISALIGNED;
+  if (int64_t(B) * int64_t(T) > kMaxM) return MLA_ERR_SHAPE;
+  const size_t need = mla_attn_oproj_fp8_workspace_bytes(B, T, mask != nullptr);
+  if (!workspace || workspace_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t M = int64_t(B) * T;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* attn = ws;
+  uint8_t* attn_q = attn + round_up(size_t(M) * MLA_OPROJ_IN * 2, 256);
+  float* attn_scale =
+      reinterpret_cast<float*>(attn_q + round_up(size_t(M) * MLA_OPROJ_IN, 256));
+  void* cls = mask ? reinterpret_cast<uint8_t*>(attn_scale) +
+                         round_up(size_t(M) * MLA_FP8_K_GROUPS * 4, 256)
+                   : nullptr;
+  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale, cls,
+                    attn, st);
+  if (s != MLA_OK) return s;
+  s = from_cuda(launch_quant_rows_fp8(attn, MLA_OPROJ_IN, M, MLA_OPROJ_IN, attn_q, attn_scale,
+                                      st));
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_fp8(attn_q, attn_scale, W_q, W_scale, out, M, MLA_HIDDEN,
+                                    MLA_OPROJ_IN, device_sm_count(), wait_limit_ns(),
+                                    device_error_word(), st));
 }
 
 mla_status_t mla_device_status(mla_stream_t stream, uint32_t* detail) {

@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 2
+    assert lib.mla_abi_version() == 3
     for code, name in binding.STATUS.items():
         assert lib.mla_status_string(code).decode() == name
     assert lib.mla_status_string(12345).decode() == "MLA_ERR_UNKNOWN"
@@ -145,6 +145,48 @@ def test_varlen_argument_errors(lib):
     assert fused_varlen(lib, ws=A + 8) == MISALIGNED
 
 
+def fused_fp8(lib, q=A, qp=A, k=A, kp=A, v=A, mask=None, ld=0, B=1, T=64, scale=0.07, Wq=A,
+              Ws=A, ws=A, ws_bytes=1 << 40, out=A):
+    return lib.mla_attn_oproj_fp8(q, qp, k, kp, v, mask, ld, B, T, scale, Wq, Ws, ws, ws_bytes,
+                                  out, None)
+
+
+def test_fp8_workspace_sizes(lib):
+    M = 4096
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, M, 0) == M * 8192 * 2 + M * 8192 + 64 * M * 4
+    # 3 tokens: 49152 + 24576 + 768, each already a multiple of 256; mask classes 1 -> 256
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 0) == 49152 + 24576 + 768
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 1) == 49152 + 24576 + 768 + 256
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(0, 3, 0) == 0
+
+
+def test_fp8_argument_errors(lib):
+    assert lib.mla_quantize_act_fp8(None, 4, A, A, None) == INVALID
+    assert lib.mla_quantize_act_fp8(A, 4, None, A, None) == INVALID
+    assert lib.mla_quantize_act_fp8(A, 4, A, None, None) == INVALID
+    assert lib.mla_quantize_act_fp8(A, 0, A, A, None) == SHAPE
+    assert lib.mla_quantize_act_fp8(A, 1 << 31, A, A, None) == SHAPE
+    assert lib.mla_quantize_act_fp8(A + 8, 4, A, A, None) == MISALIGNED
+    assert lib.mla_quantize_act_fp8(A, 4, A + 4, A, None) == MISALIGNED
+    assert lib.mla_quantize_act_fp8(A, 4, A, A + 2, None) == MISALIGNED
+    assert lib.mla_quantize_weight_fp8(None, A, A, None) == INVALID
+    assert lib.mla_quantize_weight_fp8(A, A + 8, A, None) == MISALIGNED
+    assert lib.mla_quantize_weight_fp8(A, A, A + 1, None) == MISALIGNED
+    assert lib.mla_o_proj_fp8(None, A, A, A, 4, A, None) == INVALID
+    assert lib.mla_o_proj_fp8(A, A, A, None, 4, A, None) == INVALID
+    assert lib.mla_o_proj_fp8(A, A, A, A, 0, A, None) == SHAPE
+    assert lib.mla_o_proj_fp8(A + 8, A, A, A, 4, A, None) == MISALIGNED
+    assert lib.mla_o_proj_fp8(A, A + 2, A, A, 4, A, None) == MISALIGNED
+    assert lib.mla_o_proj_fp8(A, A, A, A, 4, A + 2, None) == MISALIGNED
+    assert fused_fp8(lib, Wq=None) == INVALID
+    assert fused_fp8(lib, Ws=None) == INVALID
+    assert fused_fp8(lib, B=0) == SHAPE
+    assert fused_fp8(lib, Wq=A + 8) == MISALIGNED
+    assert fused_fp8(lib, ws=None) == WORKSPACE
+    assert fused_fp8(lib, ws_bytes=64 * 8192 * 3 + 64 * 64 * 4 - 1) == WORKSPACE
+    assert fused_fp8(lib, ws=A + 8) == MISALIGNED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path only")
 def test_valid_call_without_device_reports_cuda_error(lib):
     """With no usable device a well-formed call fails cleanly (MLA_ERR_CUDA)
@@ -152,6 +194,8 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     assert prefill(lib) in (CUDA, UNSUPPORTED)
     assert lib.mla_o_proj(A, A, 4, A, None) in (CUDA, UNSUPPORTED)
     assert varlen(lib) in (CUDA, UNSUPPORTED)
+    assert lib.mla_o_proj_fp8(A, A, A, A, 4, A, None) in (CUDA, UNSUPPORTED)
+    assert lib.mla_quantize_act_fp8(A, 4, A, A, None) in (CUDA, UNSUPPORTED)
 
 
 def test_binding_refuses_missing_library(tmp_path):
