@@ -6,11 +6,22 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/mla.h"
 
 namespace mla {
 namespace abi {
+
+// NVTX range named after the entry point, open for the call's duration, so a
+// profiler's timeline shows which library call enqueued which kernels. With
+// no tool attached the push and pop do nothing.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 constexpr int kMaxB = 65535;
 constexpr int kMaxT = 65535 * 128;

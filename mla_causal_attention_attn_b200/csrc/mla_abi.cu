@@ -126,6 +126,7 @@ mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
                               const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
                               int T, float softmax_scale, void* workspace,
                               size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_prefill");
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
                                    softmax_scale, out);
   if (s != MLA_OK) return s;
@@ -141,6 +142,7 @@ mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
 
 mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, mla_bf16* out,
                         mla_stream_t stream) {
+  CallRange range("mla_o_proj");
   if (!attn || !W_o || !out) return MLA_ERR_INVALID_ARG;
   if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
   if (!aligned16(attn) || !aligned16(W_o) || !aligned16(out)) return MLA_ERR_MISALIGNED;
@@ -164,6 +166,7 @@ mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
                             const mla_bf16* v, const mla_bf16* mask, int64_t mask_ld, int B,
                             int T, float softmax_scale, const mla_bf16* W_o, void* workspace,
                             size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_oproj");
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
                                    softmax_scale, out);
   if (s != MLA_OK) return s;
@@ -192,6 +195,7 @@ mla_status_t mla_attn_prefill_varlen(const mla_bf16* q_nope, const mla_bf16* q_p
                                      const mla_bf16* k_nope, const mla_bf16* k_pe_shared,
                                      const mla_bf16* v, const int32_t* valid_len, int B, int T,
                                      float softmax_scale, mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_prefill_varlen");
   if (!valid_len) return MLA_ERR_INVALID_ARG;
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T,
                                    softmax_scale, out);
@@ -208,6 +212,7 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                    const mla_bf16* v, const int32_t* valid_len, int B, int T,
                                    float softmax_scale, const mla_bf16* W_o, void* workspace,
                                    size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_oproj_varlen");
   if (!valid_len || !W_o) return MLA_ERR_INVALID_ARG;
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T,
                                    softmax_scale, out);
@@ -231,6 +236,7 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
 
 mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, float* scale,
                                   mla_stream_t stream) {
+  CallRange range("mla_quantize_act_fp8");
   if (!x || !q || !scale) return MLA_ERR_INVALID_ARG;
   if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
   if (!aligned16(x) || !aligned16(q) || !aligned4(scale)) return MLA_ERR_MISALIGNED;
@@ -242,6 +248,7 @@ mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, floa
 
 mla_status_t mla_quantize_weight_fp8(const mla_bf16* W, uint8_t* q, float* scale,
                                      mla_stream_t stream) {
+  CallRange range("mla_quantize_weight_fp8");
   if (!W || !q || !scale) return MLA_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(q) || !aligned4(scale)) return MLA_ERR_MISALIGNED;
   mla_status_t s = check_device();
@@ -253,6 +260,7 @@ mla_status_t mla_quantize_weight_fp8(const mla_bf16* W, uint8_t* q, float* scale
 mla_status_t mla_o_proj_fp8(const uint8_t* attn_q, const float* attn_scale, const uint8_t* W_q,
                             const float* W_scale, int64_t M, mla_bf16* out,
                             mla_stream_t stream) {
+  CallRange range("mla_o_proj_fp8");
   if (!attn_q || !attn_scale || !W_q || !W_scale || !out) return MLA_ERR_INVALID_ARG;
   if (M < 1 || M > kMaxM) return MLA_ERR_SHAPE;
   if (!aligned16(attn_q) || !aligned16(W_q) || !aligned16(out) || !aligned4(attn_scale) ||
@@ -280,6 +288,7 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                 int T, float softmax_scale, const uint8_t* W_q,
                                 const float* W_scale, void* workspace, size_t workspace_bytes,
                                 mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_oproj_fp8");
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
                                    softmax_scale, out);
   if (s != MLA_OK) return s;

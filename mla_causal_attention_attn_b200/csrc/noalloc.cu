@@ -58,6 +58,7 @@ extern "C" mla_status_t mla_attn_oproj_noalloc(const mla_bf16* q_nope, const mla
                                                const mla_bf16* mask, int64_t mask_ld, int B,
                                                int T, float softmax_scale, const mla_bf16* W_o,
                                                mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_oproj_noalloc");
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
                                    softmax_scale, out);
   if (s != MLA_OK) return s;
