@@ -72,3 +72,19 @@ def test_reference_arm_other_ranks_do_nothing(capsys):
         steps, warmup = 1, 3
     bench.run_reference(A(), None, rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+def test_fp8_oproj_flag_host_logic():
+    """--oproj fp8 names the FP8 o_proj in the config, and is refused for
+    the compact-mask workload (no fused FP8 varlen call) and the reference
+    arm."""
+    import subprocess
+    import sys
+    from mla_causal_attention_attn_b200 import inputs
+    w = inputs.WORKLOADS["b1_t4096_causal"]
+    assert "e4m3" in bench.workload_config(w, oproj="fp8")["o_proj"]
+    assert bench.workload_config(w)["o_proj"] == "8192 -> 7168"
+    for extra in (["--workload", "b8_t4096_keypad_varlen"], ["--impl", "reference"]):
+        r = subprocess.run([sys.executable, bench.__file__, "--oproj", "fp8"] + extra,
+                           capture_output=True, text=True, timeout=120)
+        assert r.returncode == 2 and "--oproj fp8" in r.stderr, r.stderr
