@@ -25,14 +25,26 @@
  *    aligned (TMA), the mask 2-byte aligned; otherwise MLA_ERR_MISALIGNED.
  *  - Streams: work is enqueued on `stream` (a cudaStream_t; NULL = legacy
  *    default stream) and the call returns without synchronising. Only
- *    mla_device_status() synchronises.
+ *    mla_last_device_status() and mla_device_status() synchronise.
  *  - Errors: every argument is checked before anything is launched; errors
  *    are returned, never thrown or printed. A kernel that gives up on an
- *    internal bounded wait records MLA_ERR_TIMEOUT in a device status word that
- *    mla_device_status() reads.
+ *    internal bounded wait records MLA_ERR_TIMEOUT in a status word instead of
+ *    trapping:
+ *      - calls given a workspace use the first word of it (the workspace
+ *        starts with MLA_WORKSPACE_STATUS_BYTES reserved for this). The call
+ *        clears that word on its stream before its kernels run, so it holds
+ *        this call's outcome alone; read it with mla_last_device_status();
+ *      - calls without a workspace (mla_o_proj, mla_attn_prefill with
+ *        workspace NULL, mla_attn_prefill_varlen, the FP8 quantisers and
+ *        GEMM, mla_attn_oproj_noalloc) use one device-wide word per device,
+ *        read and cleared atomically by mla_device_status().
  *  - Device: compute capability 10.0 (B200, sm_100a) only; otherwise
  *    MLA_ERR_UNSUPPORTED_DEVICE.
- *  - Threads: calls are thread-safe; the library holds no per-call state.
+ *  - Threads: calls are thread-safe. Mutable state shared between calls: the
+ *    device-wide status word above (calls without a workspace on different
+ *    streams report into the same word) and the no-alloc call's fixed
+ *    scratch. Cached per device and context: the SM count, device addresses
+ *    of the library's module variables, kernel attributes.
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
@@ -44,7 +56,7 @@
 extern "C" {
 #endif
 
-#define MLA_ABI_VERSION 3
+#define MLA_ABI_VERSION 4
 
 /* Model dimensions (fixed at compile time; no other values are accepted). */
 #define MLA_NUM_HEADS 64
@@ -53,6 +65,9 @@ extern "C" {
 #define MLA_V_DIM 128
 #define MLA_OPROJ_IN 8192 /* MLA_NUM_HEADS * MLA_V_DIM */
 #define MLA_HIDDEN 7168
+
+/* Bytes at the start of every workspace reserved for the call's status word. */
+#define MLA_WORKSPACE_STATUS_BYTES 256
 
 typedef uint16_t mla_bf16; /* bit pattern of a bfloat16 value */
 struct CUstream_st;
@@ -70,9 +85,9 @@ typedef enum mla_status {
 } mla_status_t;
 
 /*
- * Workspace bytes mla_attn_prefill needs: 0 when has_mask == 0; otherwise
- * B * ceil(T/128)^2 bytes for the per-tile mask classes. Returns 0 for B < 1
- * or T < 1.
+ * Workspace bytes of mla_attn_prefill: MLA_WORKSPACE_STATUS_BYTES for the
+ * call's status word, plus B * ceil(T/128)^2 bytes for the per-tile mask
+ * classes when has_mask != 0. Returns 0 for B < 1 or T < 1.
  */
 size_t mla_attn_prefill_workspace_bytes(int B, int T, int has_mask);
 
@@ -99,8 +114,11 @@ size_t mla_attn_prefill_workspace_bytes(int B, int T, int has_mask);
  *   B, T         batch (1..65535) and sequence length (1..8388480); keys = queries = T
  *   softmax_scale  multiplies Q.K^T before the mask is added (finite)
  *   workspace    device scratch of mla_attn_prefill_workspace_bytes(B,T,mask!=NULL)
- *                bytes; may be NULL when mask is NULL. Contents on entry are
- *                ignored; the call must not overlap another call using it.
+ *                bytes; required with a mask, optional (NULL) without one.
+ *                Contents on entry are ignored; the call must not overlap
+ *                another call using it. With a workspace, timeouts are
+ *                reported in it (mla_last_device_status), without one in the
+ *                device-wide word (mla_device_status).
  *   out          [B, T, 8192]: out[b,i,h*128+e], bf16
  */
 mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
@@ -123,9 +141,10 @@ mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, ml
                         mla_stream_t stream);
 
 /*
- * Workspace bytes mla_attn_oproj needs: B*T*8192*2 bytes for the merged
- * attention output, rounded up to 256, plus the mask-class bytes when
- * has_mask != 0. Returns 0 for B < 1 or T < 1.
+ * Workspace bytes mla_attn_oproj needs: MLA_WORKSPACE_STATUS_BYTES for the
+ * call's status word, B*T*8192*2 bytes for the merged attention output,
+ * rounded up to 256, plus the mask-class bytes when has_mask != 0. Returns 0
+ * for B < 1 or T < 1.
  */
 size_t mla_attn_oproj_workspace_bytes(int B, int T, int has_mask);
 
@@ -263,10 +282,10 @@ mla_status_t mla_o_proj_fp8(const uint8_t* attn_q, const float* attn_scale, cons
                             const float* W_scale, int64_t M, mla_bf16* out, mla_stream_t stream);
 
 /*
- * Workspace bytes mla_attn_oproj_fp8 needs: the merged bf16 attention output
- * (B*T*8192*2), its codes (B*T*8192) and scales (64*B*T*4), each rounded up
- * to 256, plus the mask-class bytes when has_mask != 0. Returns 0 for B < 1
- * or T < 1.
+ * Workspace bytes mla_attn_oproj_fp8 needs: MLA_WORKSPACE_STATUS_BYTES for the
+ * call's status word, the merged bf16 attention output (B*T*8192*2), its codes
+ * (B*T*8192) and scales (64*B*T*4), each rounded up to 256, plus the
+ * mask-class bytes when has_mask != 0. Returns 0 for B < 1 or T < 1.
  */
 size_t mla_attn_oproj_fp8_workspace_bytes(int B, int T, int has_mask);
 
@@ -283,11 +302,28 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                 mla_bf16* out, mla_stream_t stream);
 
 /*
- * Synchronises `stream`, then reads and clears the device status word of the
- * current device. Returns MLA_ERR_TIMEOUT if any kernel of this library gave
- * up on a bounded wait since the last call, MLA_ERR_CUDA if the stream
- * reports an error, else MLA_OK. If `detail` is not NULL it receives the raw
- * status word (kernel id << 8 | wait site, timeout flag in bit 16).
+ * Outcome of the last call that used `workspace` (a workspace given to
+ * mla_attn_prefill, mla_attn_oproj, mla_attn_oproj_varlen or
+ * mla_attn_oproj_fp8; that call must have been enqueued on `stream` or be
+ * complete). Synchronises `stream`, then reads the call's status word.
+ * Returns MLA_ERR_TIMEOUT if one of that call's kernels gave up on a bounded
+ * wait, MLA_ERR_CUDA if the stream reports an error, MLA_ERR_INVALID_ARG for
+ * a NULL workspace, MLA_ERR_MISALIGNED for one not 16-byte aligned, else
+ * MLA_OK. The word is not cleared (the next call using the workspace clears
+ * it). If `detail` is not NULL it receives the raw word (kernel id << 8 | wait
+ * site, timeout flag in bit 16; 0 when nothing was recorded).
+ */
+mla_status_t mla_last_device_status(const void* workspace, mla_stream_t stream,
+                                    uint32_t* detail);
+
+/*
+ * Synchronises `stream`, then takes the device-wide status word of the
+ * current device (the one the calls without a workspace report to): reads and
+ * clears it in one atomic step on the device, so a timeout recorded meanwhile
+ * by a kernel on another stream is kept for the next read, never lost.
+ * Returns MLA_ERR_TIMEOUT if such a kernel gave up on a bounded wait since the
+ * word was last taken, MLA_ERR_CUDA if the stream reports an error, else
+ * MLA_OK. If `detail` is not NULL it receives the raw word, as above.
  */
 mla_status_t mla_device_status(mla_stream_t stream, uint32_t* detail);
 

@@ -33,6 +33,7 @@ STATUS = {
     -7: "MLA_ERR_TIMEOUT",
 }
 MLA_OK = 0
+WORKSPACE_STATUS_BYTES = 256  # MLA_WORKSPACE_STATUS_BYTES: the status word's block
 
 # Every symbol include/mla.h declares, with its ctypes signature.
 _VP = ctypes.c_void_p
@@ -62,6 +63,7 @@ _SIGNATURES = {
     "mla_attn_oproj_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_float, _VP, _VP,
                                           _VP, ctypes.c_size_t, _VP, _VP]),
+    "mla_last_device_status": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_device_status": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_abi_version": (ctypes.c_int, []),
@@ -159,8 +161,10 @@ def attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask=None, softmax_scale=None, o
     if out is None:
         out = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=q_nope.device)
     _req(out, (B, T, K_OPROJ), "out")
-    need = attn_prefill_workspace_bytes(B, T, mask is not None)
-    if need and workspace is None:
+    # Without a mask the workspace is optional (timeouts then go to the
+    # device-wide status word); with one it holds the mask-tile classes.
+    if mask is not None and workspace is None:
+        need = attn_prefill_workspace_bytes(B, T, True)
         workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.mla_attn_prefill(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
@@ -397,8 +401,21 @@ def attn_oproj_fp8(q_nope, q_pe, k_nope, k_pe, v, W_q, W_scale, mask=None, softm
 
 
 def device_status(stream=None):
-    """Synchronise the stream; return (status, raw status word)."""
+    """Synchronise the stream; take the device-wide status word (the one the
+    calls without a workspace report to). Returns (status, raw word)."""
     lib = load()
     detail = ctypes.c_uint32(0)
     st = lib.mla_device_status(_stream_handle(stream), ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+def last_device_status(workspace, stream=None):
+    """Synchronise the stream; return (status, raw word) of the last call that
+    used ``workspace`` (``mla_last_device_status``)."""
+    lib = load()
+    if workspace is None or not workspace.is_cuda:
+        raise TypeError("workspace must be a CUDA tensor")
+    detail = ctypes.c_uint32(0)
+    st = lib.mla_last_device_status(_ptr(workspace), _stream_handle(stream),
+                                    ctypes.byref(detail))
     return int(st), int(detail.value)

@@ -27,15 +27,23 @@ constexpr int kMaxB = 65535;
 constexpr int kMaxT = 65535 * 128;
 constexpr int64_t kMaxM = (int64_t(1) << 31) - 129;
 
-// Device address of the library's status word on the current device (fetched
-// once per device), or null.
+// Device address of the device-wide status word on the current device and
+// context (looked up once per context), or null. Calls without a workspace
+// report bounded-wait timeouts there.
 unsigned int* device_error_word();
+
+// The status word a call reports timeouts to: the first word of its workspace
+// (cleared on `stream` first, so it describes this call alone) or, without a
+// workspace, the device-wide word. *st is MLA_ERR_CUDA if the clear could not
+// be enqueued.
+unsigned int* call_status_word(void* workspace, cudaStream_t stream, mla_status_t* st);
 
 // Per-wait limit of the kernels' bounded waits (MLA_WAIT_LIMIT_NS, else 1 s).
 unsigned long long wait_limit_ns();
 
 // MLA_TEST_STALL_WAIT (failure-detection tests only): 1 stalls the attention
-// kernel, 2 the small-M o_proj; 0 when unset.
+// kernel, 2 the small-M o_proj, 3 the attention kernel of masked calls only;
+// 0 when unset.
 int test_stall_wait();
 
 bool aligned16(const void* p);
@@ -53,12 +61,14 @@ mla_status_t check_attn_args(const void* q_nope, const void* q_pe, const void* k
 mla_status_t from_cuda(cudaError_t e);
 
 // Mask-tile classification (when mask is given, into `cls`) followed by the
-// attention kernel writing the merged heads to `out`. valid_len (device [B],
-// only without mask) selects causal attention with key padding.
+// attention kernel writing the merged heads to `out`; timeouts go to
+// err_word. valid_len (device [B], only without mask) selects causal
+// attention with key padding.
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
-                           cudaStream_t stream, const int* valid_len = nullptr);
+                           cudaStream_t stream, unsigned int* err_word,
+                           const int* valid_len = nullptr);
 
 }  // namespace abi
 }  // namespace mla

@@ -916,7 +916,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
       !make_map_3d(&tmV, v, kDV, T, BH, 64))
     return cudaErrorInvalidValue;
   auto kern = mask ? mla_attn_prefill_kernel<true> : mla_attn_prefill_kernel<false>;
-  static unsigned attr_done[2] = {0, 0};
+  static ContextCache attr_done[2];
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemBytes),
                                    &attr_done[mask ? 1 : 0]);
   if (e != cudaSuccess) return e;

@@ -38,6 +38,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "../../include/mla.h"
 #include "host_util.h"
 #include "sm100.cuh"
 
@@ -180,6 +181,11 @@ constexpr int kThreads = 64 + 32 * kPromoWarps;
 constexpr uint32_t kABytes = kBM * kGroup;
 constexpr int kGroupM = 16;          // row blocks visited together (L2 reuse)
 constexpr int kScaleAhead = 4;       // groups of scales loaded ahead
+// The promotion loop walks the K groups kScaleAhead at a time, so the
+// launcher needs K to be a multiple of kGroup * kScaleAhead; the o_proj
+// width (8192 input features) is one.
+static_assert(MLA_OPROJ_IN % (kGroup * kScaleAhead) == 0,
+              "o_proj input width must be a multiple of the promotion step");
 
 template <int BN>
 struct Fp8Cfg {
@@ -468,7 +474,7 @@ cudaError_t launch_fp8_bn(const CUtensorMap& tmA, const void* qw, const float* a
   const uint32_t b_box[2] = {kGroup, BN};
   if (!encode_tmap_u8(&tmB, qw, 2, b_dims, strides, b_box, true)) return cudaErrorInvalidValue;
   auto kern = oproj_fp8_kernel<BN>;
-  static unsigned attr_done = 0;
+  static ContextCache attr_done;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
                                    &attr_done);
   if (e != cudaSuccess) return e;

@@ -101,14 +101,64 @@ int device_cc() {
 
 namespace mla {
 
-cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask) {
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn get_ctx_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+std::mutex g_cache_mu;
+
+}  // namespace
+
+void* current_context() {
+  CtxGetCurrentFn fn = get_ctx_fn();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return static_cast<void*>(c);
+}
+
+void* symbol_address_cached(ContextCache* cache, const void* symbol) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= ContextCache::kMaxDevices)
+    return nullptr;
+  std::lock_guard<std::mutex> g(g_cache_mu);
+  void* ctx = current_context();
+  if (ctx && cache->ctx[dev] == ctx && cache->value[dev]) return cache->value[dev];
+  void* a = nullptr;
+  if (cudaGetSymbolAddress(&a, symbol) != cudaSuccess || a == nullptr) return nullptr;
+  // the lookup makes the device's primary context current if none was
+  cache->ctx[dev] = current_context();
+  cache->value[dev] = a;
+  return a;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes, ContextCache* done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const unsigned bit = dev < 32 ? (1u << dev) : 0u;
-  if (bit && (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  const bool cacheable = dev >= 0 && dev < ContextCache::kMaxDevices;
+  if (cacheable) {
+    std::lock_guard<std::mutex> g(g_cache_mu);
+    void* ctx = current_context();
+    if (ctx && done->ctx[dev] == ctx) return cudaSuccess;
+  }
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+  if (e == cudaSuccess && cacheable) {
+    std::lock_guard<std::mutex> g(g_cache_mu);
+    done->ctx[dev] = current_context();
+  }
   return e;
 }
 

@@ -26,8 +26,26 @@ int device_sm_count();
 // Compute capability major*10+minor of the current device (cached).
 int device_cc();
 
-// Sets the max-dynamic-shared-memory attribute of `func` once per device
-// (one bit of *done_mask per device ordinal).
-cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned* done_mask);
+// Opaque handle of the calling thread's current CUDA context (the driver's
+// CUcontext), or null if none is current or the driver entry point is missing.
+void* current_context();
+
+// Per-device cache of values that belong to one CUDA context (device
+// addresses of module variables, function attributes already set). An entry
+// is valid only for the context it was filled in: after a device reset, or
+// when another context of the same device is current, it is filled again.
+struct ContextCache {
+  static constexpr int kMaxDevices = 64;
+  void* ctx[kMaxDevices] = {};
+  void* value[kMaxDevices] = {};
+};
+
+// Device address of the module variable `symbol` on the current device and
+// context (cudaGetSymbolAddress), cached in `cache`; null if the lookup fails.
+void* symbol_address_cached(ContextCache* cache, const void* symbol);
+
+// Sets the max-dynamic-shared-memory attribute of `func` once per device and
+// context.
+cudaError_t ensure_smem_attr(const void* func, int bytes, ContextCache* done);
 
 }  // namespace mla

@@ -3,6 +3,7 @@
 // caller's stream.
 #include <cmath>
 #include <cstdlib>
+#include <mutex>
 
 #include "../../include/mla.h"
 #include "abi_internal.h"
@@ -14,26 +15,38 @@
 
 namespace mla {
 
-// The library's device status word (one per device that loads the library).
+// The device-wide status word (one per device that loads the library), used by
+// the calls that take no workspace; and the mailbox mla_device_status reads it
+// through.
 __device__ unsigned int g_device_error = 0;
+__device__ unsigned int g_status_mailbox = 0;
+
+namespace {
+
+// Takes the device-wide word and clears it in one atomic step, so that a
+// timeout recorded by a kernel on another stream meanwhile is never lost.
+__global__ void take_status_kernel(unsigned int* word, unsigned int* mailbox) {
+  *mailbox = atomicExch(word, 0u);
+}
+
+ContextCache g_error_word_cache, g_mailbox_cache;
+std::mutex g_status_mu;
+
+}  // namespace
 
 namespace abi {
 
-// Device address of g_device_error for the current device, fetched once per
-// device; null if the runtime cannot provide it.
 unsigned int* device_error_word() {
-  constexpr int kMaxDev = 64;
-  static unsigned int* addr[kMaxDev] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-  unsigned int* p = __atomic_load_n(&addr[dev], __ATOMIC_ACQUIRE);
-  if (!p) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
-    p = static_cast<unsigned int*>(a);
-    __atomic_store_n(&addr[dev], p, __ATOMIC_RELEASE);
-  }
-  return p;
+  return static_cast<unsigned int*>(
+      symbol_address_cached(&g_error_word_cache, reinterpret_cast<const void*>(&g_device_error)));
+}
+
+unsigned int* call_status_word(void* workspace, cudaStream_t stream, mla_status_t* st) {
+  *st = MLA_OK;
+  if (!workspace) return device_error_word();
+  if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), stream) != cudaSuccess)
+    *st = MLA_ERR_CUDA;
+  return static_cast<unsigned int*>(workspace);
 }
 
 unsigned long long wait_limit_ns() {
@@ -54,11 +67,12 @@ unsigned long long wait_limit_ns() {
 // to check that the kernel gives up cleanly and MLA_ERR_TIMEOUT is reported:
 // 1 = the attention kernel's first CTA waits on a barrier that nothing
 // completes; 2 = in the first cluster of the small-M o_proj, the rank-1 CTA
-// never reports its partial sum. Never set in normal use.
+// never reports its partial sum; 3 = as 1, but only in attention calls given
+// an explicit mask. Never set in normal use.
 int test_stall_wait() {
   static const int v = [] {
     const char* s = std::getenv("MLA_TEST_STALL_WAIT");
-    if (s && (s[0] == '1' || s[0] == '2') && s[1] == '\0') return s[0] - '0';
+    if (s && s[0] >= '1' && s[0] <= '3' && s[1] == '\0') return s[0] - '0';
     return 0;
   }();
   return v;
@@ -97,15 +111,17 @@ mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
-                           cudaStream_t stream, const int* valid_len) {
+                           cudaStream_t stream, unsigned int* err_word, const int* valid_len) {
   if (mask) {
     mla_status_t s = from_cuda(launch_mask_classify(mask, mask_ld, B, T, cls, stream));
     if (s != MLA_OK) return s;
   }
+  const int stall = test_stall_wait();
   return from_cuda(launch_attn_prefill(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld,
                                        mask ? cls : nullptr, B, T, softmax_scale, out,
-                                       wait_limit_ns(), device_error_word(),
-                                       test_stall_wait() == 1 ? 1 : 0, stream, valid_len));
+                                       wait_limit_ns(), err_word,
+                                       (stall == 1 || (stall == 3 && mask)) ? 1 : 0, stream,
+                                       valid_len));
 }
 
 }  // namespace abi
@@ -118,7 +134,7 @@ extern "C" {
 
 size_t mla_attn_prefill_workspace_bytes(int B, int T, int has_mask) {
   if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
-  return has_mask ? attn_class_bytes(B, T) : 0;
+  return MLA_WORKSPACE_STATUS_BYTES + (has_mask ? attn_class_bytes(B, T) : 0);
 }
 
 mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
@@ -130,14 +146,20 @@ mla_status_t mla_attn_prefill(const mla_bf16* q_nope, const mla_bf16* q_pe,
   mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T,
                                    softmax_scale, out);
   if (s != MLA_OK) return s;
-  if (mask) {
-    if (!workspace || workspace_bytes < attn_class_bytes(B, T)) return MLA_ERR_WORKSPACE;
+  if (mask && !workspace) return MLA_ERR_WORKSPACE;
+  if (workspace) {
+    if (workspace_bytes < mla_attn_prefill_workspace_bytes(B, T, mask != nullptr))
+      return MLA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
   }
   s = check_device();
   if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
+  void* cls = workspace ? static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES : nullptr;
   return run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale,
-                       workspace, out, reinterpret_cast<cudaStream_t>(stream));
+                       cls, out, st, err);
 }
 
 mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, mla_bf16* out,
@@ -156,7 +178,7 @@ mla_status_t mla_o_proj(const mla_bf16* attn, const mla_bf16* W_o, int64_t M, ml
 
 size_t mla_attn_oproj_workspace_bytes(int B, int T, int has_mask) {
   if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
-  size_t bytes = round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
+  size_t bytes = MLA_WORKSPACE_STATUS_BYTES + round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
   if (has_mask) bytes += round_up(attn_class_bytes(B, T), 256);
   return bytes;
 }
@@ -179,16 +201,17 @@ mla_status_t mla_attn_oproj(const mla_bf16* q_nope, const mla_bf16* q_pe,
   s = check_device();
   if (s != MLA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
   const size_t attn_bytes = round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
   void* attn = ws;
   void* cls = mask ? ws + attn_bytes : nullptr;
   s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale, cls,
-                    attn, st);
+                    attn, st, err);
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
-                                     device_sm_count(), wait_limit_ns(), 0, device_error_word(),
-                                     st));
+                                     device_sm_count(), wait_limit_ns(), 0, err, st));
 }
 
 mla_status_t mla_attn_prefill_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
@@ -204,7 +227,8 @@ mla_status_t mla_attn_prefill_varlen(const mla_bf16* q_nope, const mla_bf16* q_p
   s = check_device();
   if (s != MLA_OK) return s;
   return run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale,
-                       nullptr, out, reinterpret_cast<cudaStream_t>(stream), valid_len);
+                       nullptr, out, reinterpret_cast<cudaStream_t>(stream), device_error_word(),
+                       valid_len);
 }
 
 mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
@@ -226,12 +250,14 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
   s = check_device();
   if (s != MLA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale, nullptr,
-                    workspace, st, valid_len);
+  unsigned int* err = call_status_word(workspace, st, &s);
   if (s != MLA_OK) return s;
-  return from_cuda(launch_oproj_gemm(workspace, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
-                                     device_sm_count(), wait_limit_ns(), 0, device_error_word(),
-                                     st));
+  void* attn = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
+  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale, nullptr,
+                    attn, st, err, valid_len);
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, err, st));
 }
 
 mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, float* scale,
@@ -276,7 +302,8 @@ mla_status_t mla_o_proj_fp8(const uint8_t* attn_q, const float* attn_scale, cons
 size_t mla_attn_oproj_fp8_workspace_bytes(int B, int T, int has_mask) {
   if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
   const size_t M = size_t(B) * size_t(T);
-  size_t bytes = round_up(M * MLA_OPROJ_IN * 2, 256) + round_up(M * MLA_OPROJ_IN, 256) +
+  size_t bytes = MLA_WORKSPACE_STATUS_BYTES + round_up(M * MLA_OPROJ_IN * 2, 256) +
+                 round_up(M * MLA_OPROJ_IN, 256) +
                  round_up(M * MLA_FP8_K_GROUPS * 4, 256);
   if (has_mask) bytes += round_up(attn_class_bytes(B, T), 256);
   return bytes;
@@ -301,8 +328,10 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
   s = check_device();
   if (s != MLA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
   const int64_t M = int64_t(B) * T;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
   uint8_t* attn = ws;
   uint8_t* attn_q = attn + round_up(size_t(M) * MLA_OPROJ_IN * 2, 256);
   float* attn_scale =
@@ -311,29 +340,47 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
                          round_up(size_t(M) * MLA_FP8_K_GROUPS * 4, 256)
                    : nullptr;
   s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale, cls,
-                    attn, st);
+                    attn, st, err);
   if (s != MLA_OK) return s;
   s = from_cuda(launch_quant_rows_fp8(attn, MLA_OPROJ_IN, M, MLA_OPROJ_IN, attn_q, attn_scale,
                                       st));
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_fp8(attn_q, attn_scale, W_q, W_scale, out, M, MLA_HIDDEN,
-                                    MLA_OPROJ_IN, device_sm_count(), wait_limit_ns(),
-                                    device_error_word(), st));
+                                    MLA_OPROJ_IN, device_sm_count(), wait_limit_ns(), err, st));
 }
 
 mla_status_t mla_device_status(mla_stream_t stream, uint32_t* detail) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (detail) *detail = 0;
   if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
-  unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+  std::lock_guard<std::mutex> lock(g_status_mu);  // one mailbox per device
+  unsigned int* word = device_error_word();
+  unsigned int* box = static_cast<unsigned int*>(
+      symbol_address_cached(&g_mailbox_cache, reinterpret_cast<const void*>(&g_status_mailbox)));
+  if (!word || !box) return MLA_ERR_CUDA;
+  take_status_kernel<<<1, 1, 0, st>>>(word, box);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyAsync(&v, box, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
     return MLA_ERR_CUDA;
-  if (word != 0) {
-    const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
-      return MLA_ERR_CUDA;
-  }
-  if (detail) *detail = word;
-  return (word & kErrTimeoutFlag) ? MLA_ERR_TIMEOUT : MLA_OK;
+  if (detail) *detail = v;
+  return (v & kErrTimeoutFlag) ? MLA_ERR_TIMEOUT : MLA_OK;
+}
+
+mla_status_t mla_last_device_status(const void* workspace, mla_stream_t stream,
+                                    uint32_t* detail) {
+  if (detail) *detail = 0;
+  if (!workspace) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (detail) *detail = v;
+  return (v & kErrTimeoutFlag) ? MLA_ERR_TIMEOUT : MLA_OK;
 }
 
 const char* mla_status_string(mla_status_t status) {

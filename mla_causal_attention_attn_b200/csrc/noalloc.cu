@@ -4,8 +4,6 @@
 // or a plugin that is handed its inputs and outputs and nothing else. Its
 // scratch (the merged attention output and the mask-tile classes) lives in a
 // fixed, file-scope device array instead of a caller workspace.
-#include <mutex>
-
 #include "../../include/mla.h"
 #include "abi_internal.h"
 #include "attn_prefill.h"
@@ -28,22 +26,15 @@ static_assert(kAttnBytes % 256 == 0, "class region alignment");
 // the device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current) and cached; null if the lookup fails.
+// Device address of g_noalloc_scratch on the current device, looked up with
+// that device current (cudaGetSymbolAddress) and cached per device and
+// context: after a device reset, or under another context of the device, it
+// is looked up again. Null if the lookup fails.
+ContextCache g_scratch_cache;
+
 uint8_t* scratch_on_current_device() {
-  constexpr int kMaxDev = 64;
-  static std::mutex mu;
-  static uint8_t* addr[kMaxDev] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return nullptr;
-    addr[dev] = static_cast<uint8_t*>(p);
-  }
-  return addr[dev];
+  return static_cast<uint8_t*>(symbol_address_cached(
+      &g_scratch_cache, reinterpret_cast<const void*>(&g_noalloc_scratch)));
 }
 
 }  // namespace
@@ -78,7 +69,7 @@ extern "C" mla_status_t mla_attn_oproj_noalloc(const mla_bf16* q_nope, const mla
   void* attn = scratch;
   void* cls = mask ? scratch + kAttnBytes : nullptr;
   s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale, cls,
-                    attn, st);
+                    attn, st, device_error_word());
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
                                      device_sm_count(), wait_limit_ns(), 0, device_error_word(),

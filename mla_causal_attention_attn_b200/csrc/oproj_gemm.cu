@@ -275,7 +275,7 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, i
   const uint32_t box[2] = {kBK, BN};
   if (!encode_tmap_bf16(&tmB, W, 2, dims, strides, box, true)) return cudaErrorInvalidValue;
   auto kern = oproj_gemm_kernel<BN, STAGES, MT>;
-  static unsigned attr_done = 0;  // one bit per device ordinal
+  static ContextCache attr_done;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
                                    &attr_done);
   if (e != cudaSuccess) return e;
@@ -485,8 +485,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
     }
   }
 
+  // Exit rule: neither CTA leaves while its peer may still touch its shared
+  // memory (rank 1 arriving on rank 0's part_ready, rank 0 reading rank 1's
+  // partial or arriving on its part_done). After a timeout on either side
+  // those accesses can still come late, so both CTAs meet here first. Every
+  // wait above is bounded, so every thread of both CTAs reaches this barrier.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
@@ -508,7 +513,7 @@ cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M
       !encode_tmap_bf16(&tmW, W, 2, w_dims, strides, w_box, true))
     return cudaErrorInvalidValue;
   auto kern = oproj_small_m_kernel<NM, STAGES>;
-  static unsigned attr_done = 0;
+  static ContextCache attr_done;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
                                    &attr_done);
   if (e != cudaSuccess) return e;

@@ -15,9 +15,11 @@
 namespace mla {
 
 // ------------------------------------------------------------------ errors
-// Every kernel receives a pointer to the library's device-side status word. A
+// Every kernel receives a pointer to a device-side status word: the first word
+// of the call's workspace, or the device-wide word for calls without one. A
 // kernel that gives up on a wait writes a non-zero code there (first writer
-// wins) and returns; the host reads and clears it with mla_device_status().
+// wins) and returns; the host reads it with mla_last_device_status() or
+// mla_device_status().
 enum : unsigned int {
   kErrSiteMask = 0xffu,
   kErrKernelOproj = 1u << 8,
@@ -162,8 +164,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 
 // Every thread of every CTA of the cluster arrives and waits (release /
-// acquire at cluster scope). Used once, right after the barriers are
-// initialised, before any CTA touches another CTA's shared memory.
+// acquire at cluster scope). Used right after the barriers are initialised,
+// before any CTA touches another CTA's shared memory, and again before the
+// CTAs exit, so that none leaves while a peer may still access its shared
+// memory.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile(
       "barrier.cluster.arrive.release.aligned;\n\t"

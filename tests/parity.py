@@ -4,10 +4,17 @@ Tolerance (stated for the path): relative Frobenius error <= 1e-2 and max abs
 error <= 3e-2 on the bf16 outputs. Where |oracle| >= 8 the bf16 grid itself is
 coarser than 3e-2 (half an ulp is 2^-5 = 0.03125 on [8, 16)), so such
 elements are reported on their own and pass when their error is within half
-an ulp of the bf16 grid at that magnitude plus HAZARD_SLACK (the kernel's own
-pre-rounding error); the Frobenius bound is never relaxed.
+an ulp of the bf16 grid at that magnitude plus HAZARD_SLACK = 1e-3, the
+representation-limited bound; the Frobenius bound is never relaxed.
+
+With MLA_PARITY_LOG set to a file path, every check appends its label and
+metrics to that file as one JSON line (the record of n_hazard,
+hazard_worst_excess and hazard_max_err_ulps behind a run).
 """
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 import torch
@@ -15,7 +22,7 @@ import torch
 REL_FROB = 1e-2
 MAX_ABS = 3e-2
 HAZARD = 8.0
-HAZARD_SLACK = 3e-3
+HAZARD_SLACK = 1e-3
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
@@ -51,8 +58,16 @@ def metrics(got: np.ndarray, ref: np.ndarray) -> dict:
     return out
 
 
+def log_metrics(label: str, m: dict) -> None:
+    path = os.environ.get("MLA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"label": label, **m}) + "\n")
+
+
 def assert_parity(got, ref, label: str = "") -> dict:
     m = metrics(got, ref)
+    log_metrics(label, m)
     msg = f"{label}: {m}"
     assert m["finite"], msg
     assert m["rel_frob"] <= REL_FROB, msg

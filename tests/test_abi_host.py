@@ -49,21 +49,25 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.mla_abi_version() == 3
+    assert lib.mla_abi_version() == 4
     for code, name in binding.STATUS.items():
         assert lib.mla_status_string(code).decode() == name
     assert lib.mla_status_string(12345).decode() == "MLA_ERR_UNKNOWN"
 
 
+ST = binding.WORKSPACE_STATUS_BYTES  # the status word's block at the start of a workspace
+
+
 def test_workspace_sizes(lib):
-    assert lib.mla_attn_prefill_workspace_bytes(1, 4096, 0) == 0
-    assert lib.mla_attn_prefill_workspace_bytes(8, 4096, 1) == 8 * 32 * 32
-    assert lib.mla_attn_prefill_workspace_bytes(2, 129, 1) == 2 * 2 * 2
+    assert ST == 256
+    assert lib.mla_attn_prefill_workspace_bytes(1, 4096, 0) == ST
+    assert lib.mla_attn_prefill_workspace_bytes(8, 4096, 1) == ST + 8 * 32 * 32
+    assert lib.mla_attn_prefill_workspace_bytes(2, 129, 1) == ST + 2 * 2 * 2
     assert lib.mla_attn_prefill_workspace_bytes(0, 10, 1) == 0
     attn = 1 * 4096 * 8192 * 2
-    assert lib.mla_attn_oproj_workspace_bytes(1, 4096, 0) == attn
-    assert lib.mla_attn_oproj_workspace_bytes(8, 4096, 1) == 8 * 4096 * 8192 * 2 + 8 * 32 * 32
-    assert lib.mla_attn_oproj_workspace_bytes(1, 3, 0) == 49152  # 3*8192*2 rounded to 256
+    assert lib.mla_attn_oproj_workspace_bytes(1, 4096, 0) == ST + attn
+    assert lib.mla_attn_oproj_workspace_bytes(8, 4096, 1) == ST + 8 * 4096 * 8192 * 2 + 8 * 32 * 32
+    assert lib.mla_attn_oproj_workspace_bytes(1, 3, 0) == ST + 49152  # 3*8192*2 rounded to 256
     assert lib.mla_attn_oproj_workspace_bytes(-1, 3, 0) == 0
 
 
@@ -88,13 +92,15 @@ def test_prefill_argument_errors(lib):
     assert prefill(lib, T=-5) == SHAPE
     assert prefill(lib, B=65536) == SHAPE
     assert prefill(lib, T=65535 * 128 + 1) == SHAPE
-    assert prefill(lib, mask=A, ld=32, T=64, ws=A, ws_bytes=64) == SHAPE  # ld < T
+    assert prefill(lib, mask=A, ld=32, T=64, ws=A, ws_bytes=ST + 64) == SHAPE  # ld < T
     assert prefill(lib, q=A + 8) == MISALIGNED
     assert prefill(lib, v=A + 2) == MISALIGNED
     assert prefill(lib, out=A + 4) == MISALIGNED
-    assert prefill(lib, mask=A + 1, ld=64, ws=A, ws_bytes=64) == MISALIGNED  # odd address
+    assert prefill(lib, mask=A + 1, ld=64, ws=A, ws_bytes=ST + 64) == MISALIGNED  # odd address
     assert prefill(lib, mask=A, ld=64) == WORKSPACE                       # none given
-    assert prefill(lib, mask=A, ld=304, B=2, T=300, ws=A, ws_bytes=17) == WORKSPACE  # need 18
+    assert prefill(lib, mask=A, ld=304, B=2, T=300, ws=A, ws_bytes=ST + 17) == WORKSPACE  # 18
+    assert prefill(lib, ws=A, ws_bytes=ST - 1) == WORKSPACE  # optional, but then whole
+    assert prefill(lib, ws=A + 8, ws_bytes=ST) == MISALIGNED
 
 
 def test_oproj_argument_errors(lib):
@@ -114,9 +120,9 @@ def test_fused_argument_errors(lib):
     assert fused(lib, B=0) == SHAPE
     assert fused(lib, W=A + 2) == MISALIGNED
     assert fused(lib, ws=None) == WORKSPACE
-    assert fused(lib, ws_bytes=64 * 8192 * 2 - 1) == WORKSPACE
+    assert fused(lib, ws_bytes=ST + 64 * 8192 * 2 - 1) == WORKSPACE
     assert fused(lib, ws=A + 8) == MISALIGNED
-    assert fused(lib, mask=A, ld=64, ws_bytes=64 * 8192 * 2) == WORKSPACE  # class bytes missing
+    assert fused(lib, mask=A, ld=64, ws_bytes=ST + 64 * 8192 * 2) == WORKSPACE  # no class bytes
 
 
 def varlen(lib, q=A, qp=A, k=A, kp=A, v=A, vl=A, B=1, T=64, scale=0.07, out=A):
@@ -141,7 +147,7 @@ def test_varlen_argument_errors(lib):
     assert fused_varlen(lib, W=A + 2) == MISALIGNED
     assert fused_varlen(lib, vl=A + 1) == MISALIGNED
     assert fused_varlen(lib, ws=None) == WORKSPACE
-    assert fused_varlen(lib, ws_bytes=64 * 8192 * 2 - 1) == WORKSPACE
+    assert fused_varlen(lib, ws_bytes=ST + 64 * 8192 * 2 - 1) == WORKSPACE
     assert fused_varlen(lib, ws=A + 8) == MISALIGNED
 
 
@@ -153,10 +159,11 @@ def fused_fp8(lib, q=A, qp=A, k=A, kp=A, v=A, mask=None, ld=0, B=1, T=64, scale=
 
 def test_fp8_workspace_sizes(lib):
     M = 4096
-    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, M, 0) == M * 8192 * 2 + M * 8192 + 64 * M * 4
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, M, 0) == \
+        ST + M * 8192 * 2 + M * 8192 + 64 * M * 4
     # 3 tokens: 49152 + 24576 + 768, each already a multiple of 256; mask classes 1 -> 256
-    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 0) == 49152 + 24576 + 768
-    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 1) == 49152 + 24576 + 768 + 256
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 0) == ST + 49152 + 24576 + 768
+    assert lib.mla_attn_oproj_fp8_workspace_bytes(1, 3, 1) == ST + 49152 + 24576 + 768 + 256
     assert lib.mla_attn_oproj_fp8_workspace_bytes(0, 3, 0) == 0
 
 
@@ -183,8 +190,16 @@ def test_fp8_argument_errors(lib):
     assert fused_fp8(lib, B=0) == SHAPE
     assert fused_fp8(lib, Wq=A + 8) == MISALIGNED
     assert fused_fp8(lib, ws=None) == WORKSPACE
-    assert fused_fp8(lib, ws_bytes=64 * 8192 * 3 + 64 * 64 * 4 - 1) == WORKSPACE
+    assert fused_fp8(lib, ws_bytes=ST + 64 * 8192 * 3 + 64 * 64 * 4 - 1) == WORKSPACE
     assert fused_fp8(lib, ws=A + 8) == MISALIGNED
+
+
+def test_last_device_status_argument_errors(lib):
+    """The per-call status read checks its workspace before any CUDA call."""
+    detail = ctypes.c_uint32(123)
+    assert lib.mla_last_device_status(None, None, ctypes.byref(detail)) == INVALID
+    assert detail.value == 0
+    assert lib.mla_last_device_status(A + 4, None, None) == MISALIGNED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path only")

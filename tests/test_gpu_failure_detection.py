@@ -8,6 +8,8 @@ free its tensor memory and return; mla_device_status must report
 MLA_ERR_TIMEOUT with the attention kernel's code and the wait site; and the
 context must stay usable (a following o_proj call is checked against the
 oracle). Both variables are read once per process, so this runs in a child.
+The same hooks check that a timeout lands in the status word of the call that
+had it (its workspace) and nowhere else.
 """
 import json
 import os
@@ -129,3 +131,71 @@ def test_cluster_handoff_wait_times_out_and_context_survives():
     assert r["status2"] == 0, r
     assert r["attn_rel"] <= 1e-2 and r["attn_abs"] <= 3e-2, r
     assert r["oproj_rel"] <= 1e-2 and r["oproj_abs"] <= 3e-2, r
+
+
+CHILD_PER_CALL = r"""
+import json, sys
+sys.path.insert(0, ROOT)
+sys.path.insert(0, ROOT + "/tests")
+import numpy as np, torch
+import oracle
+from mla_causal_attention_attn_b200 import binding, inputs
+from parity import metrics, to_f64
+dev = torch.device("cuda:0")
+d = inputs.make_inputs(1, 512, seed=6, key_padding=True, min_valid=300)
+g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+ws_a = torch.empty(binding.attn_oproj_workspace_bytes(1, 512, True), dtype=torch.uint8, device=dev)
+ws_b = torch.empty(binding.attn_oproj_workspace_bytes(1, 512, False), dtype=torch.uint8,
+                   device=dev)
+ws_a.fill_(0xff)   # a stale word from "an earlier call" must not leak into this one
+torch.cuda.synchronize()
+args = (g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"], g["W_o"])
+# stream A: the masked call, whose first attention CTA stalls until its wait runs out
+out_a = binding.attn_oproj(*args, mask=g["mask"], softmax_scale=g["softmax_scale"],
+                           workspace=ws_a, stream=sa)
+# stream B, meanwhile: a causal call on its own workspace
+out_b = binding.attn_oproj(*args, mask=None, softmax_scale=g["softmax_scale"], workspace=ws_b,
+                           stream=sb)
+st_a, word_a = binding.last_device_status(ws_a, sa)
+st_b, word_b = binding.last_device_status(ws_b, sb)
+st_g, word_g = binding.device_status()           # the device-wide word saw nothing
+# the same workspace, next call (causal, no stall): its word starts clean
+out_a2 = binding.attn_oproj(*args, mask=None, softmax_scale=g["softmax_scale"], workspace=ws_a,
+                            stream=sa)
+st_a2, word_a2 = binding.last_device_status(ws_a, sa)
+torch.cuda.synchronize()
+ref, _ = oracle.attn_oproj_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], None,
+                                d["softmax_scale"], d["W_o"])
+mb = metrics(to_f64(out_b).reshape(512, -1), ref)
+ma2 = metrics(to_f64(out_a2).reshape(512, -1), ref)
+print(json.dumps({"st_a": st_a, "word_a": word_a, "st_b": st_b, "word_b": word_b, "st_g": st_g,
+                  "word_g": word_g, "st_a2": st_a2, "word_a2": word_a2,
+                  "b_rel": mb["rel_frob"], "b_abs": mb["max_abs"],
+                  "a2_rel": ma2["rel_frob"], "a2_abs": ma2["max_abs"]}))
+"""
+
+
+def test_status_word_is_per_workspace():
+    """Two fused calls on two streams with two workspaces. With
+    MLA_TEST_STALL_WAIT=3 only the call given an explicit mask stalls: its
+    workspace reports MLA_ERR_TIMEOUT (attention kernel), the other call's
+    workspace and the device-wide word report MLA_OK, the unaffected call's
+    output matches the oracle, and the next call on the timed-out workspace
+    starts from a clean word."""
+    env = dict(os.environ)
+    env["MLA_TEST_STALL_WAIT"] = "3"
+    env["MLA_WAIT_LIMIT_NS"] = "200000000"
+    code = "ROOT = %r\n" % ROOT + CHILD_PER_CALL
+    res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         timeout=600)
+    assert res.returncode == 0, res.stderr[-3000:]
+    r = json.loads(res.stdout.strip().splitlines()[-1])
+    assert r["st_a"] == -7, r                        # MLA_ERR_TIMEOUT, in A's workspace
+    assert r["word_a"] & (1 << 16), r
+    assert (r["word_a"] >> 8) & 0xFF == 2, r         # attention kernel
+    assert r["st_b"] == 0 and r["word_b"] == 0, r
+    assert r["st_g"] == 0 and r["word_g"] == 0, r
+    assert r["st_a2"] == 0 and r["word_a2"] == 0, r
+    assert r["b_rel"] <= 1e-2 and r["b_abs"] <= 3e-2, r
+    assert r["a2_rel"] <= 1e-2 and r["a2_abs"] <= 3e-2, r

@@ -3,20 +3,20 @@ device memory (a host framework that owns every device allocation, a plugin
 handed only its inputs and outputs). It uses the library's own fixed scratch
 instead of a caller workspace.
 
-Its output must match mla_attn_oproj (the call with a workspace) within the
-parity tolerance, on two calls in a row: the scratch is shared by every call
-and keeps the previous call's contents, so the second call must not see the
-first one's data. This file sorts last so that, if it fails, a run stopped
-at the first failure has already run every other test.
+Both calls run the same kernels on the same inputs, so the no-alloc output
+must equal mla_attn_oproj's (the call with a workspace) bit for bit, on
+several calls in a row: the scratch is shared by every call and keeps the
+previous call's contents, so a later call must not see an earlier one's data,
+and any aliasing or stale-contents mistake shows as a changed bit. This file
+sorts last so that, if it fails, a run stopped at the first failure has
+already run every other test.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
 from mla_causal_attention_attn_b200 import binding, inputs
-from parity import assert_parity, to_f64
 
 OK, WORKSPACE = 0, -5
 A = 0x7f0000000000  # 16-byte aligned fake device address (never dereferenced)
@@ -51,6 +51,10 @@ def test_noalloc_matches_workspace_call_twice_in_a_row(cuda_device):
         inputs.make_inputs(2, 300, seed=31, key_padding=True, min_valid=40),
         # causal, 8 query tiles
         inputs.make_inputs(1, 1024, seed=32),
+        # B*T <= 128: o_proj runs the small-M cluster kernel on the scratch
+        inputs.make_inputs(1, 64, seed=33),
+        # the first case again, after the scratch held the others
+        inputs.make_inputs(2, 300, seed=31, key_padding=True, min_valid=40),
     ]
     for k, d in enumerate(cases):
         g = {n: (t.to(cuda_device) if isinstance(t, torch.Tensor) else t) for n, t in d.items()}
@@ -64,7 +68,5 @@ def test_noalloc_matches_workspace_call_twice_in_a_row(cuda_device):
         torch.cuda.synchronize()
         status, word = binding.device_status()
         assert status == OK, f"device status {status} ({word:#x})"
-        got = to_f64(out).reshape(B * T, -1)
-        want = to_f64(ref).reshape(B * T, -1)
-        assert np.isfinite(got).all()
-        assert_parity(got, want, f"no-alloc call {k + 1} vs mla_attn_oproj")
+        assert torch.isfinite(out.float()).all(), f"call {k + 1}"
+        assert torch.equal(out, ref), f"no-alloc call {k + 1} differs from mla_attn_oproj"
