@@ -32,6 +32,20 @@ K_OPROJ = H * DV  # 8192, o_proj input width
 
 DEFAULT_SCALE = 1.0 / math.sqrt(DN + DR)
 
+# The rotary parameters of the configuration printed on "Kimi K2 · Block
+# input" (config.json: rope_theta and the rope_scaling block). They are
+# inputs of the rotary path, handed as they are to the kernels and to the
+# oracle.
+KIMI_K2_ROPE = {
+    "rope_theta": 50000.0,
+    "factor": 32.0,
+    "original_max_position_embeddings": 4096.0,
+    "beta_fast": 1.0,
+    "beta_slow": 1.0,
+    "mscale": 1.0,
+    "mscale_all_dim": 1.0,
+}
+
 
 @dataclasses.dataclass(frozen=True)
 class Workload:
@@ -108,6 +122,24 @@ def make_inputs(B: int, T: int, *, q_scale: float = 1.0, key_padding: bool = Fal
         out["mask"] = None
     out["softmax_scale"] = 1.0 / math.sqrt(Dn + Dr)
     return out
+
+
+def make_positions(B: int, T: int, kind: str = "arange", seed: int = 0) -> torch.Tensor:
+    """position_ids [B, T] int32 for the rotary path:
+    "arange"  0..T-1 in every sequence (what a None position_ids means);
+    "offset"  sequence b starts at 1000 * b + 17 (a prefill after a cached prefix);
+    "random"  independent draws from U{0 .. 2^17 - 1} (no structure at all)."""
+    if kind == "arange":
+        p = torch.arange(T, dtype=torch.int64).repeat(B, 1)
+    elif kind == "offset":
+        p = torch.arange(T, dtype=torch.int64).repeat(B, 1) + \
+            (1000 * torch.arange(B, dtype=torch.int64) + 17).view(B, 1)
+    elif kind == "random":
+        gen = torch.Generator().manual_seed(seed)
+        p = torch.randint(0, 1 << 17, (B, T), generator=gen, dtype=torch.int64)
+    else:
+        raise ValueError(kind)
+    return p.to(torch.int32).contiguous()
 
 
 def make_workload(w: Workload, seed: int = 0, with_weight: bool = True):

@@ -12,6 +12,8 @@ imports the other.
 What it follows: page "Kimi K2 · Mix and project", code excerpts
 modeling_deepseek.py 799-840 (query/key assembly, scaled scores, additive
 mask, fp32 softmax over keys, value mix) and 848-852 (head merge, o_proj);
+the rotary step of the same excerpt (rotary_emb / apply_rotary_pos_emb) with
+the YaRN parameters of the configuration printed on "Kimi K2 · Block input";
 for the FP8 o_proj, page "Kimi K2 · Transformer blocks", configuration
 excerpt (quantization_config: e4m3 codes, dynamic activation scales,
 128 x 128 weight blocks), with the readings stated in mla_oracle.c.
@@ -78,6 +80,19 @@ def _load():
             lib.mla_oracle_oproj_fp8_rows.argtypes = [
                 u8p, f32p, ctypes.c_int64, i64p, ctypes.c_int64, u8p, f32p, ctypes.c_int,
                 ctypes.c_int, f64p]
+            lib.mla_oracle_yarn_inv_freq.restype = ctypes.c_int
+            lib.mla_oracle_yarn_inv_freq.argtypes = [ctypes.c_int] + [ctypes.c_double] * 5 + [f64p]
+            lib.mla_oracle_yarn_attn_factor.restype = ctypes.c_double
+            lib.mla_oracle_yarn_attn_factor.argtypes = [ctypes.c_double] * 3
+            lib.mla_oracle_rope_rotate.restype = ctypes.c_int
+            lib.mla_oracle_rope_rotate.argtypes = [u16p, ctypes.c_int64, ctypes.c_int, i64p, f64p,
+                                                   ctypes.c_double, f64p]
+            lib.mla_oracle_attn_rows_rope.restype = ctypes.c_int
+            lib.mla_oracle_attn_rows_rope.argtypes = [
+                u16p, u16p, u16p, u16p, u16p, u16p, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, f64p, ctypes.c_double,
+                i64p, i64p, ctypes.c_int64, f64p, f64p, u8p]
             lib.mla_oracle_num_threads.restype = ctypes.c_int
             lib.mla_oracle_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -194,6 +209,108 @@ def attn_oproj_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, W_o,
     """
     attn, fm = attn_rows(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale,
                          rows=rows)
+    return oproj_rows(attn, W_o), fm.any(axis=1)
+
+
+# ------------------------------------------------------------------ rotary (YaRN)
+# The readings (pair layout, YaRN frequencies, attention factor) are stated in
+# mla_oracle.c. A parameter set is a mapping with the keys of config.json's
+# rope_scaling plus rope_theta.
+
+def yarn_inv_freq(Dr, rope) -> np.ndarray:
+    """The Dr/2 rotation frequencies (radians per position) of a YaRN set."""
+    out = np.zeros(Dr // 2, dtype=np.float64)
+    rc = _load().mla_oracle_yarn_inv_freq(
+        int(Dr), float(rope["rope_theta"]), float(rope["factor"]),
+        float(rope["original_max_position_embeddings"]), float(rope["beta_fast"]),
+        float(rope["beta_slow"]), _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle yarn_inv_freq rejected {rope}")
+    return out
+
+
+def yarn_attn_factor(rope) -> float:
+    """The factor YaRN multiplies cos and sin by."""
+    return float(_load().mla_oracle_yarn_attn_factor(
+        float(rope["factor"]), float(rope["mscale"]), float(rope["mscale_all_dim"])))
+
+
+def _positions(position_ids, B, T) -> np.ndarray:
+    if position_ids is None:
+        return np.ascontiguousarray(np.tile(np.arange(T, dtype=np.int64), B))
+    import torch
+    p = position_ids
+    if isinstance(p, torch.Tensor):
+        p = p.detach().cpu().numpy()
+    p = np.asarray(p, dtype=np.int64)
+    if p.shape != (B, T):
+        raise ValueError(f"position_ids must be [B, T] = {(B, T)}, got {p.shape}")
+    return np.ascontiguousarray(p.reshape(-1))
+
+
+def rope_rotate(x, positions, rope) -> np.ndarray:
+    """Rotated copy (float64) of bf16 rotary vectors x [..., Dr] at integer
+    positions of shape x.shape[:-1]."""
+    bits = _bf16_bits(x)
+    Dr = bits.shape[-1]
+    n = int(np.prod(bits.shape[:-1]))
+    pos = np.ascontiguousarray(np.asarray(positions, dtype=np.int64).reshape(-1))
+    if pos.shape[0] != n:
+        raise ValueError("one position per rotary vector")
+    inv = yarn_inv_freq(Dr, rope)
+    out = np.zeros((n, Dr), dtype=np.float64)
+    rc = _load().mla_oracle_rope_rotate(_ptr(bits, ctypes.c_uint16), ctypes.c_int64(n), Dr,
+                                        _ptr(pos, ctypes.c_int64), _ptr(inv, ctypes.c_double),
+                                        yarn_attn_factor(rope), _ptr(out, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle rope_rotate failed ({rc})")
+    return out.reshape(bits.shape)
+
+
+def attn_rows_rope(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, position_ids, rope,
+                   rows=None):
+    """attn_rows with q_pe and k_pe given unrotated: both are rotated (YaRN,
+    at position_ids [B, T], or 0..T-1 when None) before the scores."""
+    B, H, T, Dn = q_nope.shape
+    Dr = q_pe.shape[-1]
+    Dv = v.shape[-1]
+    if tuple(q_pe.shape) != (B, H, T, Dr) or tuple(k_pe.shape) != (B, 1, T, Dr) or \
+            tuple(k_nope.shape) != (B, H, T, Dn) or tuple(v.shape) != (B, H, T, Dv):
+        raise ValueError("input shapes do not match")
+    if mask is not None and tuple(mask.shape) != (B, 1, T, T):
+        raise ValueError("mask must be [B,1,T,T]")
+    if rows is None:
+        rb = np.repeat(np.arange(B, dtype=np.int64), T)
+        ri = np.tile(np.arange(T, dtype=np.int64), B)
+    else:
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+        rb = np.ascontiguousarray(rows[:, 0])
+        ri = np.ascontiguousarray(rows[:, 1])
+    R = rb.shape[0]
+    arrays = [_bf16_bits(t) for t in (q_nope, q_pe, k_nope, k_pe, v)]
+    m = _bf16_bits(mask) if mask is not None else None
+    pos = _positions(position_ids, B, T)
+    inv = yarn_inv_freq(Dr, rope)
+    out = np.zeros((R, H * Dv), dtype=np.float64)
+    fm = np.zeros((R, H), dtype=np.uint8)
+    scale = float(np.float32(softmax_scale))
+    rc = _load().mla_oracle_attn_rows_rope(
+        *[_ptr(a, ctypes.c_uint16) for a in arrays],
+        _ptr(m, ctypes.c_uint16) if m is not None else None,
+        ctypes.c_int64(T), B, H, T, Dn, Dr, Dv, scale, _ptr(pos, ctypes.c_int64),
+        _ptr(inv, ctypes.c_double), yarn_attn_factor(rope),
+        _ptr(rb, ctypes.c_int64), _ptr(ri, ctypes.c_int64), ctypes.c_int64(R),
+        _ptr(out, ctypes.c_double), None, _ptr(fm, ctypes.c_uint8))
+    if rc != 0:
+        raise RuntimeError(f"oracle attn_rows_rope failed ({rc})")
+    return out, fm.astype(bool)
+
+
+def attn_oproj_rows_rope(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, position_ids, rope,
+                         W_o, rows=None):
+    """Full path with unrotated q_pe / k_pe: rotation, attention, o_proj."""
+    attn, fm = attn_rows_rope(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, position_ids,
+                              rope, rows=rows)
     return oproj_rows(attn, W_o), fm.any(axis=1)
 
 

@@ -19,7 +19,8 @@
  *
  * and, for the FP8 form of o_proj (end of this file), the e4m3 codes, the
  * dynamic per-token and 128 x 128 block quantisers and the block-scaled
- * product.
+ * product; and the YaRN rotation of the rotary parts (section "rotary"),
+ * for callers that pass q_pe and k_pe unrotated.
  *
  * - The query and key of every head are the concatenation of a non-rotary
  *   part and a rotary part; the key's rotary part is one tensor shared by all
@@ -100,6 +101,16 @@ void mla_oracle_set_num_threads(int n)
  *
  * Returns 0, or -1 on an argument error.
  */
+static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
+                          const uint16_t *k_nope, const uint16_t *k_pe,
+                          const uint16_t *v, const uint16_t *mask,
+                          int64_t mask_ld, int B, int H, int T, int Dn, int Dr,
+                          int Dv, double scale, const int64_t *row_b,
+                          const int64_t *row_i, int64_t nrows, double *out,
+                          double *probs, uint8_t *fully_masked,
+                          const int64_t *pos, const double *inv_freq,
+                          double attn_factor);
+
 int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
                          const uint16_t *k_nope, const uint16_t *k_pe,
                          const uint16_t *v, const uint16_t *mask,
@@ -107,6 +118,142 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
                          int Dv, double scale, const int64_t *row_b,
                          const int64_t *row_i, int64_t nrows, double *out,
                          double *probs, uint8_t *fully_masked)
+{
+    return attn_rows_impl(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, H, T,
+                          Dn, Dr, Dv, scale, row_b, row_i, nrows, out, probs,
+                          fully_masked, NULL, NULL, 1.0);
+}
+
+/* ================================================================ rotary
+ *
+ * The rotary parts are rotated right before the query and key are assembled
+ * (page "Kimi K2 · Mix and project", excerpt modeling_deepseek.py 799-840:
+ * cos, sin = self.rotary_emb(...); apply_rotary_pos_emb(q_pe, k_pe, cos, sin,
+ * position_ids)). The pages print neither function's body. What they do
+ * print is the configuration (page "Kimi K2 · Block input", config.json):
+ * qk_rope_head_dim 64, rope_theta 50000, rope_scaling {type yarn, factor 32,
+ * original_max_position_embeddings 4096, beta_fast 1, beta_slow 1, mscale 1,
+ * mscale_all_dim 1}. The readings taken here, from the published YaRN method
+ * (Peng et al., "YaRN: Efficient Context Window Extension of Large Language
+ * Models", 2023: NTK-by-parts interpolation plus an attention factor):
+ *
+ * - Pair i (i < Dr/2) of a rotary vector is its elements 2i and 2i+1, rotated
+ *   as one complex number by the angle position * inv_freq[i]:
+ *     out[2i]   = f * (x[2i] cos a - x[2i+1] sin a)
+ *     out[2i+1] = f * (x[2i+1] cos a + x[2i] sin a)
+ *   with f the attention factor below. (An implementation may store the
+ *   rotated pair elsewhere in the vector, e.g. first halves then second
+ *   halves; as long as query and key are stored alike, every score is the
+ *   same number.)
+ * - The base frequencies are theta^(-2i/Dr). YaRN keeps them (extrapolation)
+ *   for the fast-rotating pairs and divides them by `factor` (interpolation)
+ *   for the slow ones, with a linear ramp between two pair indices:
+ *     d(n)  = Dr * ln(L / (2 pi n)) / (2 ln theta)     (L = original max positions;
+ *             the pair index that turns n times over L positions)
+ *     low   = max(floor(d(beta_fast)), 0), high = min(ceil(d(beta_slow)), Dr - 1)
+ *             (high = low + 0.001 when they coincide)
+ *     ramp  = clamp((i - low) / (high - low), 0, 1)
+ *     inv_freq[i] = theta^(-2i/Dr) * ((1 - ramp) + ramp / factor)
+ *   With the printed values (beta_fast = beta_slow = 1) low = 19, high = 20:
+ *   pairs 0..19 keep their frequency, pairs 20..31 are divided by 32.
+ * - The attention factor multiplies cos and sin:
+ *     f = m(factor, mscale) / m(factor, mscale_all_dim),
+ *     m(s, k) = 1 if s <= 1 else 0.1 k ln(s) + 1,
+ *   which is exactly 1 for the printed mscale = mscale_all_dim = 1.
+ * - Query and key rotate with the same position_ids (the excerpt passes one
+ *   position_ids to apply_rotary_pos_emb); without them positions are 0..T-1.
+ */
+
+int mla_oracle_yarn_inv_freq(int Dr, double theta, double factor,
+                             double orig_max_pos, double beta_fast,
+                             double beta_slow, double *inv_freq)
+{
+    if (Dr < 2 || (Dr & 1) || !(theta > 1.0) || !(factor > 0.0) ||
+        !(orig_max_pos > 0.0) || !(beta_fast > 0.0) || !(beta_slow > 0.0) ||
+        !inv_freq)
+        return -1;
+    const double two_pi = 2.0 * acos(-1.0);
+    const double d_fast = Dr * log(orig_max_pos / (two_pi * beta_fast)) / (2.0 * log(theta));
+    const double d_slow = Dr * log(orig_max_pos / (two_pi * beta_slow)) / (2.0 * log(theta));
+    double low = floor(d_fast), high = ceil(d_slow);
+    if (low < 0.0) low = 0.0;
+    if (high > Dr - 1) high = Dr - 1;
+    if (high == low) high += 0.001;
+    for (int i = 0; i < Dr / 2; ++i) {
+        const double base = pow(theta, -2.0 * i / Dr);
+        double ramp = (i - low) / (high - low);
+        if (ramp < 0.0) ramp = 0.0;
+        if (ramp > 1.0) ramp = 1.0;
+        inv_freq[i] = base * (1.0 - ramp) + (base / factor) * ramp;
+    }
+    return 0;
+}
+
+static double yarn_m(double s, double k)
+{
+    return s <= 1.0 ? 1.0 : 0.1 * k * log(s) + 1.0;
+}
+
+double mla_oracle_yarn_attn_factor(double factor, double mscale, double mscale_all_dim)
+{
+    return yarn_m(factor, mscale) / yarn_m(factor, mscale_all_dim);
+}
+
+/* Rotate one rotary vector of Dr bf16 values at position p (double out). */
+static void rotate_row(const uint16_t *x, int Dr, int64_t p, const double *inv_freq,
+                       double f, double *out)
+{
+    for (int i = 0; i < Dr / 2; ++i) {
+        const double a = (double)p * inv_freq[i];
+        const double c = f * cos(a), sn = f * sin(a);
+        const double x0 = bf16_bits_to_double(x[2 * i]);
+        const double x1 = bf16_bits_to_double(x[2 * i + 1]);
+        out[2 * i] = x0 * c - x1 * sn;
+        out[2 * i + 1] = x1 * c + x0 * sn;
+    }
+}
+
+/* Rotated copies of n rotary vectors x [n, Dr] at positions pos[n]. */
+int mla_oracle_rope_rotate(const uint16_t *x, int64_t n, int Dr, const int64_t *pos,
+                           const double *inv_freq, double attn_factor, double *out)
+{
+    if (n < 0 || Dr < 2 || (Dr & 1) || (n > 0 && (!x || !pos || !inv_freq || !out)))
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        rotate_row(x + r * Dr, Dr, pos[r], inv_freq, attn_factor, out + r * Dr);
+    return 0;
+}
+
+/*
+ * mla_oracle_attn_rows with the rotary parts given unrotated: q_pe and k_pe
+ * are rotated here (as above) at positions pos [B, T] before the scores.
+ */
+int mla_oracle_attn_rows_rope(const uint16_t *q_nope, const uint16_t *q_pe,
+                              const uint16_t *k_nope, const uint16_t *k_pe,
+                              const uint16_t *v, const uint16_t *mask,
+                              int64_t mask_ld, int B, int H, int T, int Dn, int Dr,
+                              int Dv, double scale, const int64_t *pos,
+                              const double *inv_freq, double attn_factor,
+                              const int64_t *row_b, const int64_t *row_i,
+                              int64_t nrows, double *out, double *probs,
+                              uint8_t *fully_masked)
+{
+    if (!pos || !inv_freq || Dr < 2 || (Dr & 1)) return -1;
+    return attn_rows_impl(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, H, T,
+                          Dn, Dr, Dv, scale, row_b, row_i, nrows, out, probs,
+                          fully_masked, pos, inv_freq, attn_factor);
+}
+
+static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
+                          const uint16_t *k_nope, const uint16_t *k_pe,
+                          const uint16_t *v, const uint16_t *mask,
+                          int64_t mask_ld, int B, int H, int T, int Dn, int Dr,
+                          int Dv, double scale, const int64_t *row_b,
+                          const int64_t *row_i, int64_t nrows, double *out,
+                          double *probs, uint8_t *fully_masked,
+                          const int64_t *pos, const double *inv_freq,
+                          double attn_factor)
 {
     if (B < 1 || H < 1 || T < 1 || Dn < 0 || Dr < 0 || Dv < 1 || nrows < 0)
         return -1;
@@ -119,6 +266,14 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
     for (int64_t r = 0; r < nrows; ++r)
         if (row_b[r] < 0 || row_b[r] >= B || row_i[r] < 0 || row_i[r] >= T)
             return -1;
+
+    /* the shared rotary key, rotated once for every (b, j) when rotating */
+    double *k_rot = NULL;
+    if (pos && Dr > 0) {
+        k_rot = (double *)malloc(sizeof(double) * (size_t)B * (size_t)T * (size_t)Dr);
+        if (!k_rot) return -2;
+        mla_oracle_rope_rotate(k_pe, (int64_t)B * T, Dr, pos, inv_freq, attn_factor, k_rot);
+    }
 
     const int64_t work = nrows * (int64_t)H;
     int bad_alloc = 0;
@@ -146,8 +301,12 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
             /* the query row, non-rotary part then rotary part */
             for (int d = 0; d < Dn; ++d)
                 qv[d] = bf16_bits_to_double(q_nope[(bh * T + i) * Dn + d]);
-            for (int d = 0; d < Dr; ++d)
-                qv[Dn + d] = bf16_bits_to_double(q_pe[(bh * T + i) * Dr + d]);
+            if (k_rot)
+                rotate_row(q_pe + (bh * T + i) * Dr, Dr, pos[b * T + i], inv_freq,
+                           attn_factor, qv + Dn);
+            else
+                for (int d = 0; d < Dr; ++d)
+                    qv[Dn + d] = bf16_bits_to_double(q_pe[(bh * T + i) * Dr + d]);
 
             /* pass 1: every score of the row, and its maximum */
             double smax = -INFINITY;
@@ -165,8 +324,12 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
                     double dot = 0.0;
                     for (int d = 0; d < Dn; ++d)
                         dot += qv[d] * bf16_bits_to_double(k_nope[(bh * T + j) * Dn + d]);
-                    for (int d = 0; d < Dr; ++d)
-                        dot += qv[Dn + d] * bf16_bits_to_double(k_pe[(b * T + j) * Dr + d]);
+                    if (k_rot)
+                        for (int d = 0; d < Dr; ++d)
+                            dot += qv[Dn + d] * k_rot[(b * T + j) * Dr + d];
+                    else
+                        for (int d = 0; d < Dr; ++d)
+                            dot += qv[Dn + d] * bf16_bits_to_double(k_pe[(b * T + j) * Dr + d]);
                     sj = scale * dot + add;
                 }
                 s[j] = sj;
@@ -209,6 +372,7 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
         free(qv);
         free(acc);
     }
+    free(k_rot);
     return bad_alloc ? -2 : 0;
 }
 
