@@ -191,6 +191,96 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                    float softmax_scale, const mla_bf16* W_o, void* workspace,
                                    size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
 
+/*
+ * ------------------------------------------------------------ rotary inputs
+ * The excerpt rotates the rotary parts right before assembling query and key
+ * (page "Kimi K2 · Mix and project", excerpt modeling_deepseek.py 799-840:
+ * cos, sin = self.rotary_emb(value_states, ...); q_pe, k_pe =
+ * apply_rotary_pos_emb(q_pe, k_pe, cos, sin, position_ids)). The calls below
+ * take q_pe and k_pe unrotated and do that step themselves, with the YaRN
+ * rotary embedding whose parameters config.json prints (page "Kimi K2 · Block
+ * input": rope_theta and rope_scaling). The pages print neither function's
+ * body; the library reads them as:
+ *  - pair i (i < 32) of a rotary vector, elements 2i and 2i+1, turns as one
+ *    complex number by the angle position * inv_freq[i], and both elements
+ *    are multiplied by the attention factor f;
+ *  - inv_freq[i] = theta^(-i/32) * ((1 - r_i) + r_i / factor), r_i =
+ *    clamp((i - lo) / (hi - lo), 0, 1), with lo = floor(d(beta_fast)),
+ *    hi = ceil(d(beta_slow)) clamped to [0, 63], d(n) = 64 ln(L / (2 pi n)) /
+ *    (2 ln theta), L = original_max_position_embeddings (YaRN's NTK-by-parts
+ *    interpolation; hi = lo + 0.001 when they meet). The printed values give
+ *    lo = 19, hi = 20: pairs 0..19 keep theta^(-i/32), pairs 20..31 divide it
+ *    by 32;
+ *  - f = m(factor, mscale) / m(factor, mscale_all_dim), m(s, k) = 1 for
+ *    s <= 1, else 0.1 k ln(s) + 1 (exactly 1 for the printed values);
+ *  - query and key use the same position_ids.
+ * Angles, cos and sin are computed in double precision; the rotated values
+ * are rounded once to bf16 before the score MMAs.
+ */
+typedef struct mla_yarn_rope {
+  double rope_theta;                       /* > 1 */
+  double factor;                           /* > 0 */
+  double original_max_position_embeddings; /* > 0 */
+  double beta_fast;                        /* > 0 */
+  double beta_slow;                        /* > 0 */
+  double mscale;
+  double mscale_all_dim;
+} mla_yarn_rope_t;
+
+/* The printed configuration's values, as an initializer of mla_yarn_rope_t. */
+#define MLA_KIMI_K2_YARN_ROPE {50000.0, 32.0, 4096.0, 1.0, 1.0, 1.0, 1.0}
+
+/*
+ * Workspace bytes of mla_attn_prefill_rope: MLA_WORKSPACE_STATUS_BYTES, the
+ * rotated key (B*T*64*2) and the cos/sin table (B*T*32*8), each rounded up to
+ * 256, plus the mask-class bytes (rounded up to 256) when has_mask != 0.
+ * Returns 0 for B < 1 or T < 1.
+ */
+size_t mla_attn_prefill_rope_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * mla_attn_prefill with unrotated rotary parts:
+ *   q_pe          [B, 64, T, 64] rotary query parts before rotation
+ *   k_pe          [B, 1, T, 64]  shared rotary key before rotation
+ *   position_ids  [B, T] int32 device array (4-byte aligned), the position of
+ *                 every token; NULL means 0..T-1 in every sequence. Any int32
+ *                 value is used as given.
+ *   rope          host pointer to the rotary parameters (read during the
+ *                 call only); NULL, a non-finite value or one out of range
+ *                 -> MLA_ERR_INVALID_ARG.
+ *   workspace     mla_attn_prefill_rope_workspace_bytes(B, T, mask != NULL)
+ *                 bytes, required (it holds the rotated key and the table).
+ * Every other argument, the layouts and the errors as in mla_attn_prefill.
+ * The shared key is rotated once per call by a small pre-pass kernel; each
+ * query tile's q_pe is rotated by the attention kernel in shared memory right
+ * after its load. With all positions 0 the result equals mla_attn_prefill's
+ * on the same inputs, bit for bit.
+ */
+mla_status_t mla_attn_prefill_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* k_nope, const mla_bf16* k_pe,
+                                   const mla_bf16* v, const int32_t* position_ids,
+                                   const mla_yarn_rope_t* rope, const mla_bf16* mask,
+                                   int64_t mask_ld, int B, int T, float softmax_scale,
+                                   void* workspace, size_t workspace_bytes, mla_bf16* out,
+                                   mla_stream_t stream);
+
+/*
+ * Workspace bytes of mla_attn_oproj_rope: mla_attn_prefill_rope_workspace_bytes
+ * plus the merged attention output (B*T*8192*2, rounded up to 256).
+ */
+size_t mla_attn_oproj_rope_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * mla_attn_prefill_rope followed by o_proj, as mla_attn_oproj:
+ *   out [B, T, 7168] bf16.
+ */
+mla_status_t mla_attn_oproj_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                 const mla_bf16* k_nope, const mla_bf16* k_pe, const mla_bf16* v,
+                                 const int32_t* position_ids, const mla_yarn_rope_t* rope,
+                                 const mla_bf16* mask, int64_t mask_ld, int B, int T,
+                                 float softmax_scale, const mla_bf16* W_o, void* workspace,
+                                 size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
+
 /* Largest B*T mla_attn_oproj_noalloc accepts (its fixed scratch holds the
  * merged attention output of this many tokens: 64 MiB). */
 #define MLA_NOALLOC_MAX_TOKENS 4096
@@ -303,9 +393,9 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
 
 /*
  * Outcome of the last call that used `workspace` (a workspace given to
- * mla_attn_prefill, mla_attn_oproj, mla_attn_oproj_varlen or
- * mla_attn_oproj_fp8; that call must have been enqueued on `stream` or be
- * complete). Synchronises `stream`, then reads the call's status word.
+ * mla_attn_prefill, mla_attn_oproj, mla_attn_oproj_varlen,
+ * mla_attn_prefill_rope, mla_attn_oproj_rope or mla_attn_oproj_fp8; that call
+ * must have been enqueued on `stream` or be complete). Synchronises `stream`, then reads the call's status word.
  * Returns MLA_ERR_TIMEOUT if one of that call's kernels gave up on a bounded
  * wait, MLA_ERR_CUDA if the stream reports an error, MLA_ERR_INVALID_ARG for
  * a NULL workspace, MLA_ERR_MISALIGNED for one not 16-byte aligned, else

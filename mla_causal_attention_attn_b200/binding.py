@@ -35,8 +35,22 @@ STATUS = {
 MLA_OK = 0
 WORKSPACE_STATUS_BYTES = 256  # MLA_WORKSPACE_STATUS_BYTES: the status word's block
 
+class YarnRope(ctypes.Structure):
+    """mla_yarn_rope_t: config.json's rope_theta and rope_scaling fields."""
+    _fields_ = [("rope_theta", ctypes.c_double), ("factor", ctypes.c_double),
+                ("original_max_position_embeddings", ctypes.c_double),
+                ("beta_fast", ctypes.c_double), ("beta_slow", ctypes.c_double),
+                ("mscale", ctypes.c_double), ("mscale_all_dim", ctypes.c_double)]
+
+
+def _yarn(rope) -> YarnRope:
+    r = _inputs.KIMI_K2_ROPE if rope is None else rope
+    return YarnRope(*[float(r[f]) for f, _ in YarnRope._fields_])
+
+
 # Every symbol include/mla.h declares, with its ctypes signature.
 _VP = ctypes.c_void_p
+_ROPE_P = ctypes.POINTER(YarnRope)
 _SIGNATURES = {
     "mla_attn_prefill_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "mla_attn_prefill": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64, ctypes.c_int,
@@ -55,6 +69,16 @@ _SIGNATURES = {
     "mla_attn_oproj_varlen": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_float, _VP, _VP,
                                              ctypes.c_size_t, _VP, _VP]),
+    "mla_attn_prefill_rope_workspace_bytes": (ctypes.c_size_t,
+                                              [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_prefill_rope": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _ROPE_P, _VP,
+                                             ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_float, _VP, ctypes.c_size_t, _VP, _VP]),
+    "mla_attn_oproj_rope_workspace_bytes": (ctypes.c_size_t,
+                                            [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_oproj_rope": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _ROPE_P, _VP,
+                                           ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_float, _VP, _VP, ctypes.c_size_t, _VP, _VP]),
     "mla_quantize_act_fp8": (ctypes.c_int, [_VP, ctypes.c_int64, _VP, _VP, _VP]),
     "mla_quantize_weight_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP]),
     "mla_o_proj_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]),
@@ -272,6 +296,86 @@ def attn_oproj_varlen(q_nope, q_pe, k_nope, k_pe, v, valid_len, W_o, softmax_sca
                                    _ptr(valid_len), B, T, scale, _ptr(W_o), _ptr(workspace),
                                    ws_bytes, _ptr(out), _stream_handle(stream))
     _check("mla_attn_oproj_varlen", st)
+    return out
+
+
+def _positions(position_ids, B, T):
+    if position_ids is None:
+        return None
+    if position_ids.dtype != torch.int32 or not position_ids.is_cuda:
+        raise TypeError("position_ids must be an int32 CUDA tensor")
+    if tuple(position_ids.shape) != (B, T) or not position_ids.is_contiguous():
+        raise ValueError(f"position_ids must be a contiguous [{B}, {T}] tensor")
+    return position_ids
+
+
+def attn_prefill_rope_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_prefill_rope_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def attn_oproj_rope_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_oproj_rope_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def attn_prefill_rope(q_nope, q_pe, k_nope, k_pe, v, position_ids=None, rope=None, mask=None,
+                      softmax_scale=None, out=None, workspace=None, stream=None):
+    """Attention with unrotated q_pe / k_pe (YaRN rotation at position_ids
+    [B, T] int32, None = 0..T-1; rope = a mapping of config.json's rotary
+    fields, None = the printed Kimi K2 values), [B, T, 8192] bf16, via
+    ``mla_attn_prefill_rope``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    pos = _positions(position_ids, B, T)
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, K_OPROJ), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, K_OPROJ), "out")
+    if workspace is None:
+        workspace = torch.empty(attn_prefill_rope_workspace_bytes(B, T, mask is not None),
+                                dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    yr = _yarn(rope)
+    st = lib.mla_attn_prefill_rope(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                   _ptr(pos), ctypes.byref(yr), _ptr(mask), mask_ld, B, T, scale,
+                                   _ptr(workspace), ws_bytes, _ptr(out), _stream_handle(stream))
+    _check("mla_attn_prefill_rope", st)
+    return out
+
+
+def attn_oproj_rope(q_nope, q_pe, k_nope, k_pe, v, W_o, position_ids=None, rope=None, mask=None,
+                    softmax_scale=None, out=None, workspace=None, stream=None):
+    """Whole path with unrotated q_pe / k_pe, [B, T, 7168] bf16, via
+    ``mla_attn_oproj_rope``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(v, (B, H, T, DV), "v")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    pos = _positions(position_ids, B, T)
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    if workspace is None:
+        workspace = torch.empty(attn_oproj_rope_workspace_bytes(B, T, mask is not None),
+                                dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    yr = _yarn(rope)
+    st = lib.mla_attn_oproj_rope(_ptr(q_nope), _ptr(q_pe), _ptr(k_nope), _ptr(k_pe), _ptr(v),
+                                 _ptr(pos), ctypes.byref(yr), _ptr(mask), mask_ld, B, T, scale,
+                                 _ptr(W_o), _ptr(workspace), ws_bytes, _ptr(out),
+                                 _stream_handle(stream))
+    _check("mla_attn_oproj_rope", st)
     return out
 
 

@@ -22,7 +22,7 @@ LIB_NAME = "libmla_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
 SOURCES = ["mla_abi.cu", "attn_prefill.cu", "oproj_gemm.cu", "fp8_oproj.cu", "host_util.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "rope.cu"]
 GENCODE = "arch=compute_100a,code=sm_100a"
 
 

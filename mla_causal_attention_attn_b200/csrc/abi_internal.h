@@ -63,12 +63,13 @@ mla_status_t from_cuda(cudaError_t e);
 // Mask-tile classification (when mask is given, into `cls`) followed by the
 // attention kernel writing the merged heads to `out`; timeouts go to
 // err_word. valid_len (device [B], only without mask) selects causal
-// attention with key padding.
+// attention with key padding; rope_cs (the rotary pre-pass's cos / sin
+// table) makes the kernel rotate q_pe, with k_pe already rotated.
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
                            cudaStream_t stream, unsigned int* err_word,
-                           const int* valid_len = nullptr);
+                           const int* valid_len = nullptr, const void* rope_cs = nullptr);
 
 }  // namespace abi
 }  // namespace mla

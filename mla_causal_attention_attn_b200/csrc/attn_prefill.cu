@@ -90,6 +90,8 @@ struct AttnArgs {
   unsigned long long wait_limit_ns;
   unsigned int* err_word;      // device status word
   int test_stall;              // failure-detection test: one wait that never completes
+  const float2* rope_cs;       // [B*T][32] (f cos, f sin) of each query's rotary pairs, or
+                               // null when q_pe arrives rotated
 };
 
 // Which key tiles the two query tiles of a CTA visit. Causal: tile qt visits
@@ -260,7 +262,7 @@ __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r
   }
 }
 
-template <bool kMasked>
+template <bool kMasked, bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQn,
                             const __grid_constant__ CUtensorMap tmQp,
@@ -269,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[2];     // query tile i is in shared memory
+  __shared__ uint64_t q_rot[2];      // its rotary part is rotated (rotary calls only)
   __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
   __shared__ uint64_t s_full[2], p_full[2];
   __shared__ uint64_t o_final[2];
@@ -316,6 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_flag = 0;
     mbar_init(&q_full[0], 1);
     mbar_init(&q_full[1], 1);
+    mbar_init(&q_rot[0], 128);
+    mbar_init(&q_rot[1], 128);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&ring_full[s], 1);
       // released once by each query tile's MMA issuer
@@ -450,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t o_tmem = tmem_base + kColO + 128 * qi;
       const bool pair = tiles.exists[1];
       bool ok = mbar_wait(&q_full[qi], 0, ctl, 10);
+      if (kRope && ok) ok = mbar_wait(&q_rot[qi], 0, ctl, 16);
       bool issued_any = false;
       uint32_t n_pv = 0;       // PVs issued
       uint32_t n_tiles = 0;    // visited key tiles so far
@@ -571,9 +577,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const __nv_bfloat16* mrow =
         (kMasked && row_valid) ? args.mask + (size_t(b) * args.T + q) * args.mask_ld : nullptr;
 
+    bool ok = true;
+    if (kRope && has_work && tiles.exists[wi]) {
+      // Rotary calls: rotate this row's q_pe (64 values, the tile's third
+      // 16 KB block, 128-byte rows with the 16-byte chunks XOR-swizzled by
+      // row % 8) in shared memory once its TMA load has landed; pair i =
+      // elements 2i, 2i+1 turns by the (f cos, f sin) tabulated for this
+      // query's position. The MMA issuer waits for all 128 rows (q_rot).
+      ok = mbar_wait(&q_full[wi], 0, ctl, 24);
+      if (ok && row_valid) {
+        uint8_t* rowp = smem + kOffQ + wi * kQBytes + 2 * kBlock + r * 128;
+        const float4* cs = reinterpret_cast<const float4*>(args.rope_cs + (size_t(b) * args.T + q) * 32);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // 16-byte chunk c holds pairs 4c .. 4c+3
+          uint4* chunk = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
+          uint4 w = *chunk;
+          const float4 a = __ldg(cs + 2 * c), bq = __ldg(cs + 2 * c + 1);
+          const float csn[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = bf16_bits_to_float(wp[e] & 0xffffu);
+            const float x1 = bf16_bits_to_float(wp[e] >> 16);
+            const float cc = csn[2 * e], ss = csn[2 * e + 1];
+            wp[e] = pack_bf16x2(fmaf(x0, cc, -x1 * ss), fmaf(x1, cc, x0 * ss));
+          }
+          *chunk = w;
+        }
+        fence_proxy_async_smem();  // the MMA reads it through the async proxy
+      }
+      mbar_arrive(&q_rot[wi]);
+    }
     float m = -INFINITY;  // running max, log2 units
     float l = 0.f;        // running sum of p (fp32, unrounded)
-    bool ok = true;
     uint32_t n = 0;
     for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) {
       if (!tiles.active(wi, kt)) continue;
@@ -907,7 +943,8 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
-                                int test_stall, cudaStream_t stream, const int* valid_len) {
+                                int test_stall, cudaStream_t stream, const int* valid_len,
+                                const void* rope_cs) {
   if (mask && valid_len) return cudaErrorInvalidValue;
   CUtensorMap tmQn, tmQp, tmKn, tmKp, tmV;
   const int BH = B * kH;
@@ -915,10 +952,13 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
       !make_map_3d(&tmKn, k_nope, kDN, T, BH) || !make_map_3d(&tmKp, k_pe, kDR, T, B) ||
       !make_map_3d(&tmV, v, kDV, T, BH, 64))
     return cudaErrorInvalidValue;
-  auto kern = mask ? mla_attn_prefill_kernel<true> : mla_attn_prefill_kernel<false>;
-  static ContextCache attr_done[2];
+  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true>
+                             : mla_attn_prefill_kernel<true, false>)
+                  : (rope_cs ? mla_attn_prefill_kernel<false, true>
+                             : mla_attn_prefill_kernel<false, false>);
+  static ContextCache attr_done[4];
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemBytes),
-                                   &attr_done[mask ? 1 : 0]);
+                                   &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0)]);
   if (e != cudaSuccess) return e;
   AttnArgs a;
   a.mask = static_cast<const __nv_bfloat16*>(mask);
@@ -936,6 +976,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   a.wait_limit_ns = wait_limit_ns;
   a.err_word = err_word;
   a.test_stall = test_stall;
+  a.rope_cs = static_cast<const float2*>(rope_cs);
   const long long ctas = (long long)B * kH * a.n_pairs;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
   kern<<<unsigned(ctas), kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, a);

@@ -29,13 +29,16 @@ cudaError_t launch_mask_classify(const void* mask, int64_t mask_ld, int B, int T
 // mask == null: causal. tile_class may be null when mask is given (every key
 // tile is then visited and masked element-wise). valid_len (device, [B] int32,
 // only without mask): causal with keys j >= valid_len[b] masked (values are
-// clamped to [0, T]); null means every sequence has all T keys.
+// clamped to [0, T]); null means every sequence has all T keys. rope_cs
+// (device, [B*T][32] float2 of (f cos, f sin), from launch_rope_prepass):
+// q_pe arrives unrotated and each query tile's rotary part is rotated in
+// shared memory (k_pe must then be the rotated key); null: q_pe is rotated.
 cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void* k_nope,
                                 const void* k_pe, const void* v, const void* mask,
                                 int64_t mask_ld, const void* tile_class, int B, int T,
                                 float softmax_scale, void* out,
                                 unsigned long long wait_limit_ns, unsigned int* err_word,
                                 int test_stall, cudaStream_t stream,
-                                const int* valid_len = nullptr);
+                                const int* valid_len = nullptr, const void* rope_cs = nullptr);
 
 }  // namespace mla

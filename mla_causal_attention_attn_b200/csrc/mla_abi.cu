@@ -11,6 +11,7 @@
 #include "fp8_oproj.h"
 #include "host_util.h"
 #include "oproj_gemm.h"
+#include "rope.h"
 #include "sm100.cuh"
 
 namespace mla {
@@ -111,7 +112,8 @@ mla_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
 mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_nope,
                            const void* k_pe, const void* v, const void* mask, int64_t mask_ld,
                            int B, int T, float softmax_scale, void* cls, void* out,
-                           cudaStream_t stream, unsigned int* err_word, const int* valid_len) {
+                           cudaStream_t stream, unsigned int* err_word, const int* valid_len,
+                           const void* rope_cs) {
   if (mask) {
     mla_status_t s = from_cuda(launch_mask_classify(mask, mask_ld, B, T, cls, stream));
     if (s != MLA_OK) return s;
@@ -121,7 +123,21 @@ mla_status_t run_attention(const void* q_nope, const void* q_pe, const void* k_n
                                        mask ? cls : nullptr, B, T, softmax_scale, out,
                                        wait_limit_ns(), err_word,
                                        (stall == 1 || (stall == 3 && mask)) ? 1 : 0, stream,
-                                       valid_len));
+                                       valid_len, rope_cs));
+}
+
+mla_status_t rope_freqs(const mla_yarn_rope_t* rope, RopeFreqs* f) {
+  if (!rope) return MLA_ERR_INVALID_ARG;
+  return yarn_frequencies(rope->rope_theta, rope->factor, rope->original_max_position_embeddings,
+                          rope->beta_fast, rope->beta_slow, rope->mscale, rope->mscale_all_dim, f)
+             ? MLA_OK
+             : MLA_ERR_INVALID_ARG;
+}
+
+// Workspace regions of the rotary calls after the status block: the rotated
+// key, then the cos / sin table.
+size_t rope_region_bytes(int B, int T) {
+  return round_up(rope_krot_bytes(B, T), 256) + round_up(rope_cs_bytes(B, T), 256);
 }
 
 }  // namespace abi
@@ -255,6 +271,94 @@ mla_status_t mla_attn_oproj_varlen(const mla_bf16* q_nope, const mla_bf16* q_pe,
   void* attn = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
   s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, nullptr, 0, B, T, softmax_scale, nullptr,
                     attn, st, err, valid_len);
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, err, st));
+}
+
+size_t mla_attn_prefill_rope_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  size_t bytes = MLA_WORKSPACE_STATUS_BYTES + rope_region_bytes(B, T);
+  if (has_mask) bytes += round_up(attn_class_bytes(B, T), 256);
+  return bytes;
+}
+
+mla_status_t mla_attn_prefill_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* k_nope, const mla_bf16* k_pe,
+                                   const mla_bf16* v, const int32_t* position_ids,
+                                   const mla_yarn_rope_t* rope, const mla_bf16* mask,
+                                   int64_t mask_ld, int B, int T, float softmax_scale,
+                                   void* workspace, size_t workspace_bytes, mla_bf16* out,
+                                   mla_stream_t stream) {
+  CallRange range("mla_attn_prefill_rope");
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  RopeFreqs f;
+  s = rope_freqs(rope, &f);
+  if (s != MLA_OK) return s;
+  if (position_ids && !aligned4(position_ids)) return MLA_ERR_MISALIGNED;
+  if (!workspace ||
+      workspace_bytes < mla_attn_prefill_rope_workspace_bytes(B, T, mask != nullptr))
+    return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
+  uint8_t* k_rot = ws;
+  uint8_t* cs = k_rot + round_up(rope_krot_bytes(B, T), 256);
+  void* cls = mask ? ws + rope_region_bytes(B, T) : nullptr;
+  s = from_cuda(launch_rope_prepass(k_pe, position_ids, B, T, f, cs, k_rot, st));
+  if (s != MLA_OK) return s;
+  return run_attention(q_nope, q_pe, k_nope, k_rot, v, mask, mask_ld, B, T, softmax_scale, cls,
+                       out, st, err, nullptr, cs);
+}
+
+size_t mla_attn_oproj_rope_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  return mla_attn_prefill_rope_workspace_bytes(B, T, has_mask) +
+         round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
+}
+
+mla_status_t mla_attn_oproj_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                 const mla_bf16* k_nope, const mla_bf16* k_pe, const mla_bf16* v,
+                                 const int32_t* position_ids, const mla_yarn_rope_t* rope,
+                                 const mla_bf16* mask, int64_t mask_ld, int B, int T,
+                                 float softmax_scale, const mla_bf16* W_o, void* workspace,
+                                 size_t workspace_bytes, mla_bf16* out, mla_stream_t stream) {
+  CallRange range("mla_attn_oproj_rope");
+  mla_status_t s = check_attn_args(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if (!W_o) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_o)) return MLA_ERR_MISALIGNED;
+  if (int64_t(B) * int64_t(T) > kMaxM) return MLA_ERR_SHAPE;
+  RopeFreqs f;
+  s = rope_freqs(rope, &f);
+  if (s != MLA_OK) return s;
+  if (position_ids && !aligned4(position_ids)) return MLA_ERR_MISALIGNED;
+  if (!workspace ||
+      workspace_bytes < mla_attn_oproj_rope_workspace_bytes(B, T, mask != nullptr))
+    return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
+  // status | rotated key | cos/sin table | merged attention | mask classes
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
+  uint8_t* k_rot = ws;
+  uint8_t* cs = k_rot + round_up(rope_krot_bytes(B, T), 256);
+  uint8_t* attn = ws + rope_region_bytes(B, T);
+  void* cls = mask ? attn + round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256) : nullptr;
+  s = from_cuda(launch_rope_prepass(k_pe, position_ids, B, T, f, cs, k_rot, st));
+  if (s != MLA_OK) return s;
+  s = run_attention(q_nope, q_pe, k_nope, k_rot, v, mask, mask_ld, B, T, softmax_scale, cls,
+                    attn, st, err, nullptr, cs);
   if (s != MLA_OK) return s;
   return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
                                      device_sm_count(), wait_limit_ns(), 0, err, st));

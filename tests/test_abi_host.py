@@ -221,3 +221,36 @@ def test_binding_refuses_missing_library(tmp_path):
             binding.load(str(tmp_path / "nope.so"))
         finally:
             binding._lib = old
+
+
+def rope_call(lib, q=A, qp=A, k=A, kp=A, v=A, pos=None, rope="k2", mask=None, ld=0, B=1, T=64,
+              scale=0.07, ws=A, ws_bytes=1 << 40, out=A):
+    r = None if rope is None else ctypes.byref(
+        binding._yarn(None) if rope == "k2" else binding.YarnRope(*rope))
+    return lib.mla_attn_prefill_rope(q, qp, k, kp, v, pos, r, mask, ld, B, T, scale, ws,
+                                     ws_bytes, out, None)
+
+
+def test_rope_workspace_sizes(lib):
+    # status | rotated key (B*T*128) | cos/sin table (B*T*256) | classes
+    assert lib.mla_attn_prefill_rope_workspace_bytes(1, 4096, 0) == ST + 4096 * 128 + 4096 * 256
+    assert lib.mla_attn_prefill_rope_workspace_bytes(2, 3, 1) == ST + 768 + 1536 + 256
+    assert lib.mla_attn_oproj_rope_workspace_bytes(1, 3, 0) == ST + 512 + 768 + 49152  # 384 -> 512
+    assert lib.mla_attn_prefill_rope_workspace_bytes(0, 3, 0) == 0
+
+
+def test_rope_argument_errors(lib):
+    k2 = (50000.0, 32.0, 4096.0, 1.0, 1.0, 1.0, 1.0)
+    assert rope_call(lib, rope=None) == INVALID
+    assert rope_call(lib, rope=(1.0,) + k2[1:]) == INVALID             # theta must exceed 1
+    assert rope_call(lib, rope=k2[:1] + (0.0,) + k2[2:]) == INVALID    # factor > 0
+    assert rope_call(lib, rope=k2[:3] + (-1.0,) + k2[4:]) == INVALID   # beta_fast > 0
+    assert rope_call(lib, rope=k2[:5] + (float("nan"),) + k2[6:]) == INVALID
+    assert rope_call(lib, q=None) == INVALID
+    assert rope_call(lib, B=0) == SHAPE
+    assert rope_call(lib, pos=A + 2) == MISALIGNED
+    assert rope_call(lib, ws=None) == WORKSPACE                          # always required
+    assert rope_call(lib, ws_bytes=ST + 64 * 128 + 64 * 256 - 1) == WORKSPACE
+    assert rope_call(lib, ws=A + 8) == MISALIGNED
+    assert lib.mla_attn_oproj_rope(A, A, A, A, A, None, ctypes.byref(binding._yarn(None)), None,
+                                   0, 1, 64, 0.07, None, A, 1 << 40, A, None) == INVALID
