@@ -142,6 +142,25 @@ def make_positions(B: int, T: int, kind: str = "arange", seed: int = 0) -> torch
     return p.to(torch.int32).contiguous()
 
 
+KV_RANK = 512  # kv_lora_rank
+
+
+def make_latent_inputs(B: int, T: int, *, q_scale: float = 1.0, key_padding: bool = False,
+                       min_valid: int = 512, seed: int = 0, H_: int = H, Dn: int = DN,
+                       Dr: int = DR, Dv: int = DV, R: int = KV_RANK, D: int = D_MODEL,
+                       with_weight: bool = True):
+    """Inputs of the path that starts from the compressed KV latent: the
+    make_inputs set (whose k_nope and v are then unused), followed by draws of
+    c_kv [B, T, R] ~ N(0, 1) and W_kv_b [H*(Dn+Dv), R] ~ N(0, 0.02) (the
+    configuration's initializer_range, as for W_o)."""
+    out = make_inputs(B, T, q_scale=q_scale, key_padding=key_padding, min_valid=min_valid,
+                      seed=seed, H_=H_, Dn=Dn, Dr=Dr, Dv=Dv, D=D, with_weight=with_weight)
+    gen = torch.Generator().manual_seed(seed + 7919)
+    out["c_kv"] = _randn(gen, (B, T, R))
+    out["W_kv_b"] = _randn(gen, (H_ * (Dn + Dv), R), std=0.02)
+    return out
+
+
 def make_workload(w: Workload, seed: int = 0, with_weight: bool = True):
     return make_inputs(w.B, w.T, q_scale=w.q_scale, key_padding=w.key_padding,
                        min_valid=w.min_valid, seed=seed, with_weight=with_weight)

@@ -93,6 +93,14 @@ def _load():
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, f64p, ctypes.c_double,
                 i64p, i64p, ctypes.c_int64, f64p, f64p, u8p]
+            lib.mla_oracle_kv_up.restype = ctypes.c_int
+            lib.mla_oracle_kv_up.argtypes = [u16p, u16p] + [ctypes.c_int] * 6 + [f64p, f64p]
+            lib.mla_oracle_attn_rows_kv64.restype = ctypes.c_int
+            lib.mla_oracle_attn_rows_kv64.argtypes = [
+                u16p, u16p, f64p, u16p, f64p, u16p, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_double, i64p, i64p,
+                ctypes.c_int64, f64p, f64p, u8p]
             lib.mla_oracle_num_threads.restype = ctypes.c_int
             lib.mla_oracle_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -311,6 +319,72 @@ def attn_oproj_rows_rope(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, pos
     """Full path with unrotated q_pe / k_pe: rotation, attention, o_proj."""
     attn, fm = attn_rows_rope(q_nope, q_pe, k_nope, k_pe, v, mask, softmax_scale, position_ids,
                               rope, rows=rows)
+    return oproj_rows(attn, W_o), fm.any(axis=1)
+
+
+# ------------------------------------------------------------------ latent up-projection
+# Reading (mla_oracle.c, section "latent"): one bias-free linear map of each
+# token's latent to 64 heads x (128 non-rotary key + 128 value), the key part
+# first within each head's block of rows of W.
+
+def kv_up(c_kv, W_kv, H, Dn, Dv):
+    """k_nope [B,H,T,Dn] and v [B,H,T,Dv] (float64) from the bf16 latent
+    c_kv [B,T,R] and the bf16 weight W_kv [H*(Dn+Dv), R]."""
+    x = _bf16_bits(c_kv)
+    w = _bf16_bits(W_kv)
+    B, T, R = x.shape
+    if w.shape != (H * (Dn + Dv), R):
+        raise ValueError(f"W_kv must be [{H * (Dn + Dv)}, {R}], got {w.shape}")
+    k = np.zeros((B, H, T, Dn), dtype=np.float64)
+    v = np.zeros((B, H, T, Dv), dtype=np.float64)
+    rc = _load().mla_oracle_kv_up(_ptr(x, ctypes.c_uint16), _ptr(w, ctypes.c_uint16), B, T, R, H,
+                                  Dn, Dv, _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle kv_up failed ({rc})")
+    return k, v
+
+
+def attn_rows_kv64(q_nope, q_pe, k_nope64, k_pe, v64, mask, softmax_scale, rows=None):
+    """attn_rows with the non-rotary keys and the values given in float64."""
+    B, H, T, Dn = q_nope.shape
+    Dr = q_pe.shape[-1]
+    Dv = v64.shape[-1]
+    k_nope64 = np.ascontiguousarray(k_nope64, dtype=np.float64)
+    v64 = np.ascontiguousarray(v64, dtype=np.float64)
+    if k_nope64.shape != (B, H, T, Dn) or v64.shape[:3] != (B, H, T) or \
+            tuple(k_pe.shape) != (B, 1, T, Dr) or tuple(q_pe.shape) != (B, H, T, Dr):
+        raise ValueError("input shapes do not match")
+    if mask is not None and tuple(mask.shape) != (B, 1, T, T):
+        raise ValueError("mask must be [B,1,T,T]")
+    if rows is None:
+        rb = np.repeat(np.arange(B, dtype=np.int64), T)
+        ri = np.tile(np.arange(T, dtype=np.int64), B)
+    else:
+        rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+        rb = np.ascontiguousarray(rows[:, 0])
+        ri = np.ascontiguousarray(rows[:, 1])
+    R = rb.shape[0]
+    qn, qp, kp = (_bf16_bits(t) for t in (q_nope, q_pe, k_pe))
+    m = _bf16_bits(mask) if mask is not None else None
+    out = np.zeros((R, H * Dv), dtype=np.float64)
+    fm = np.zeros((R, H), dtype=np.uint8)
+    rc = _load().mla_oracle_attn_rows_kv64(
+        _ptr(qn, ctypes.c_uint16), _ptr(qp, ctypes.c_uint16), _ptr(k_nope64, ctypes.c_double),
+        _ptr(kp, ctypes.c_uint16), _ptr(v64, ctypes.c_double),
+        _ptr(m, ctypes.c_uint16) if m is not None else None, ctypes.c_int64(T), B, H, T, Dn, Dr,
+        Dv, float(np.float32(softmax_scale)), _ptr(rb, ctypes.c_int64), _ptr(ri, ctypes.c_int64),
+        ctypes.c_int64(R), _ptr(out, ctypes.c_double), None, _ptr(fm, ctypes.c_uint8))
+    if rc != 0:
+        raise RuntimeError(f"oracle attn_rows_kv64 failed ({rc})")
+    return out, fm.astype(bool)
+
+
+def attn_oproj_rows_latent(q_nope, q_pe, c_kv, W_kv, k_pe, mask, softmax_scale, W_o, rows=None):
+    """Full path from the latent: up-projection, attention, head merge, o_proj."""
+    H, Dn = q_nope.shape[1], q_nope.shape[3]
+    Dv = W_kv.shape[0] // H - Dn
+    k, v = kv_up(c_kv, W_kv, H, Dn, Dv)
+    attn, fm = attn_rows_kv64(q_nope, q_pe, k, k_pe, v, mask, softmax_scale, rows=rows)
     return oproj_rows(attn, W_o), fm.any(axis=1)
 
 

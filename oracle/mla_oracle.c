@@ -19,8 +19,9 @@
  *
  * and, for the FP8 form of o_proj (end of this file), the e4m3 codes, the
  * dynamic per-token and 128 x 128 block quantisers and the block-scaled
- * product; and the YaRN rotation of the rotary parts (section "rotary"),
- * for callers that pass q_pe and k_pe unrotated.
+ * product; the YaRN rotation of the rotary parts (section "rotary"), for
+ * callers that pass q_pe and k_pe unrotated; and the up-projection of the
+ * compressed KV latent into k_nope and v (section "latent").
  *
  * - The query and key of every head are the concatenation of a non-rotary
  *   part and a rotary part; the key's rotary part is one tensor shared by all
@@ -109,7 +110,8 @@ static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
                           const int64_t *row_i, int64_t nrows, double *out,
                           double *probs, uint8_t *fully_masked,
                           const int64_t *pos, const double *inv_freq,
-                          double attn_factor);
+                          double attn_factor, const double *k_nope_f64,
+                          const double *v_f64);
 
 int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
                          const uint16_t *k_nope, const uint16_t *k_pe,
@@ -121,7 +123,7 @@ int mla_oracle_attn_rows(const uint16_t *q_nope, const uint16_t *q_pe,
 {
     return attn_rows_impl(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, H, T,
                           Dn, Dr, Dv, scale, row_b, row_i, nrows, out, probs,
-                          fully_masked, NULL, NULL, 1.0);
+                          fully_masked, NULL, NULL, 1.0, NULL, NULL);
 }
 
 /* ================================================================ rotary
@@ -242,7 +244,72 @@ int mla_oracle_attn_rows_rope(const uint16_t *q_nope, const uint16_t *q_pe,
     if (!pos || !inv_freq || Dr < 2 || (Dr & 1)) return -1;
     return attn_rows_impl(q_nope, q_pe, k_nope, k_pe, v, mask, mask_ld, B, H, T,
                           Dn, Dr, Dv, scale, row_b, row_i, nrows, out, probs,
-                          fully_masked, pos, inv_freq, attn_factor);
+                          fully_masked, pos, inv_freq, attn_factor, NULL, NULL);
+}
+
+/* ================================================================ latent
+ *
+ * The non-rotary key parts and the values come from the compressed KV
+ * latent: config.json (page "Kimi K2 · Block input") gives kv_lora_rank 512,
+ * num_attention_heads 64, qk_nope_head_dim 128, v_head_dim 128 and
+ * attention_bias false, and the excerpt of page "Kimi K2 · Mix and project"
+ * starts from per-head k_nope and value_states. The pages print nothing in
+ * between; the reading taken here is the plain linear up-projection, one
+ * bias-free nn.Linear(512 -> 64 * (128 + 128)) applied to each token's
+ * latent:
+ *   kv[b,t,n] = sum_{c<R} c_kv[b,t,c] * W[n,c]                  (W [H*(Dn+Dv), R])
+ *   k_nope[b,h,t,e] = kv[b,t,h*(Dn+Dv) + e]          (e < Dn)
+ *   v[b,h,t,e]      = kv[b,t,h*(Dn+Dv) + Dn + e]     (e < Dv)
+ * i.e. the output is viewed per head as Dn + Dv values, the non-rotary key
+ * part first, then the value.
+ */
+
+/* k_nope [B,H,T,Dn] and v [B,H,T,Dv] (double) from c_kv [B,T,R] and W. */
+int mla_oracle_kv_up(const uint16_t *c_kv, const uint16_t *W, int B, int T, int R,
+                     int H, int Dn, int Dv, double *k_nope, double *v)
+{
+    if (B < 1 || T < 1 || R < 1 || H < 1 || Dn < 0 || Dv < 1 || !c_kv || !W || !v ||
+        (Dn > 0 && !k_nope))
+        return -1;
+    const int per_head = Dn + Dv;
+    const int64_t work = (int64_t)B * T * H;
+#pragma omp parallel for schedule(static)
+    for (int64_t w = 0; w < work; ++w) {
+        const int64_t bt = w / H;
+        const int h = (int)(w % H);
+        const int64_t b = bt / T, t = bt % T;
+        const uint16_t *x = c_kv + bt * R;
+        for (int n = 0; n < per_head; ++n) {
+            const uint16_t *wrow = W + ((int64_t)h * per_head + n) * R;
+            double acc = 0.0;
+            for (int c = 0; c < R; ++c)
+                acc += bf16_bits_to_double(x[c]) * bf16_bits_to_double(wrow[c]);
+            if (n < Dn)
+                k_nope[((b * H + h) * T + t) * Dn + n] = acc;
+            else
+                v[((b * H + h) * T + t) * Dv + (n - Dn)] = acc;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Attention whose non-rotary keys and values are given in double (the
+ * up-projection's exact result above) instead of bf16; q_pe, k_pe as in
+ * mla_oracle_attn_rows (rotated).
+ */
+int mla_oracle_attn_rows_kv64(const uint16_t *q_nope, const uint16_t *q_pe,
+                              const double *k_nope, const uint16_t *k_pe,
+                              const double *v, const uint16_t *mask,
+                              int64_t mask_ld, int B, int H, int T, int Dn, int Dr,
+                              int Dv, double scale, const int64_t *row_b,
+                              const int64_t *row_i, int64_t nrows, double *out,
+                              double *probs, uint8_t *fully_masked)
+{
+    if (!v || (Dn > 0 && !k_nope)) return -1;
+    return attn_rows_impl(q_nope, q_pe, NULL, k_pe, NULL, mask, mask_ld, B, H, T,
+                          Dn, Dr, Dv, scale, row_b, row_i, nrows, out, probs,
+                          fully_masked, NULL, NULL, 1.0, k_nope, v);
 }
 
 static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
@@ -253,15 +320,16 @@ static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
                           const int64_t *row_i, int64_t nrows, double *out,
                           double *probs, uint8_t *fully_masked,
                           const int64_t *pos, const double *inv_freq,
-                          double attn_factor)
+                          double attn_factor, const double *k_nope_f64,
+                          const double *v_f64)
 {
     if (B < 1 || H < 1 || T < 1 || Dn < 0 || Dr < 0 || Dv < 1 || nrows < 0)
         return -1;
     if (!q_nope && Dn > 0) return -1;
-    if (!k_nope && Dn > 0) return -1;
+    if (!k_nope && !k_nope_f64 && Dn > 0) return -1;
     if (!q_pe && Dr > 0) return -1;
     if (!k_pe && Dr > 0) return -1;
-    if (!v || !out || (nrows > 0 && (!row_b || !row_i))) return -1;
+    if ((!v && !v_f64) || !out || (nrows > 0 && (!row_b || !row_i))) return -1;
     if (mask && mask_ld < T) return -1;
     for (int64_t r = 0; r < nrows; ++r)
         if (row_b[r] < 0 || row_b[r] >= B || row_i[r] < 0 || row_i[r] >= T)
@@ -322,8 +390,12 @@ static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
                     sj = -INFINITY;
                 } else {
                     double dot = 0.0;
-                    for (int d = 0; d < Dn; ++d)
-                        dot += qv[d] * bf16_bits_to_double(k_nope[(bh * T + j) * Dn + d]);
+                    if (k_nope_f64)
+                        for (int d = 0; d < Dn; ++d)
+                            dot += qv[d] * k_nope_f64[(bh * T + j) * Dn + d];
+                    else
+                        for (int d = 0; d < Dn; ++d)
+                            dot += qv[d] * bf16_bits_to_double(k_nope[(bh * T + j) * Dn + d]);
                     if (k_rot)
                         for (int d = 0; d < Dr; ++d)
                             dot += qv[Dn + d] * k_rot[(b * T + j) * Dr + d];
@@ -362,9 +434,14 @@ static int attn_rows_impl(const uint16_t *q_nope, const uint16_t *q_pe,
                 const double p = s[j] / denom;
                 if (prow) prow[j] = p;
                 if (p == 0.0) continue;
-                const uint16_t *vrow = v + (bh * T + j) * Dv;
-                for (int e = 0; e < Dv; ++e)
-                    acc[e] += p * bf16_bits_to_double(vrow[e]);
+                if (v_f64) {
+                    const double *vrow = v_f64 + (bh * T + j) * Dv;
+                    for (int e = 0; e < Dv; ++e) acc[e] += p * vrow[e];
+                } else {
+                    const uint16_t *vrow = v + (bh * T + j) * Dv;
+                    for (int e = 0; e < Dv; ++e)
+                        acc[e] += p * bf16_bits_to_double(vrow[e]);
+                }
             }
             for (int e = 0; e < Dv; ++e) orow[e] = acc[e];
         }
