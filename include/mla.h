@@ -35,9 +35,9 @@
  *        clears that word on its stream before its kernels run, so it holds
  *        this call's outcome alone; read it with mla_last_device_status();
  *      - calls without a workspace (mla_o_proj, mla_attn_prefill with
- *        workspace NULL, mla_attn_prefill_varlen, the FP8 quantisers and
- *        GEMM, mla_attn_oproj_noalloc) use one device-wide word per device,
- *        read and cleared atomically by mla_device_status().
+ *        workspace NULL, mla_attn_prefill_varlen, mla_kv_up_proj, the FP8
+ *        quantisers and GEMM, mla_attn_oproj_noalloc) use one device-wide
+ *        word per device, read and cleared atomically by mla_device_status().
  *  - Device: compute capability 10.0 (B200, sm_100a) only; otherwise
  *    MLA_ERR_UNSUPPORTED_DEVICE.
  *  - Threads: calls are thread-safe. Mutable state shared between calls: the
@@ -281,6 +281,52 @@ mla_status_t mla_attn_oproj_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                  float softmax_scale, const mla_bf16* W_o, void* workspace,
                                  size_t workspace_bytes, mla_bf16* out, mla_stream_t stream);
 
+/*
+ * ------------------------------------------------------------ KV latent
+ * The non-rotary key parts and the values come from each token's compressed
+ * KV latent of kv_lora_rank = 512 values (config.json on page "Kimi K2 · Block
+ * input"). The pages print only the rank; the library reads the step as one
+ * bias-free linear map (attention_bias false) per token,
+ *   kv[b,t,:] = c_kv[b,t,:] . W_kv_b^T,   W_kv_b [64 * 256, 512],
+ * whose 256 outputs per head h (rows h*256 .. h*256+255 of W_kv_b) are the
+ * head's 128 non-rotary key parts followed by its 128 values.
+ */
+#define MLA_KV_RANK 512
+
+/*
+ * Up-projection of the latent into the attention's key and value layouts:
+ *   c_kv    [B, T, 512] bf16
+ *   W_kv_b  [16384, 512] bf16
+ *   k_nope  [B, 64, T, 128] bf16: k_nope[b,h,t,e] = kv[b,t,h*256 + e]
+ *   v       [B, 64, T, 128] bf16: v[b,h,t,e]      = kv[b,t,h*256 + 128 + e]
+ * fp32 accumulation, each output rounded once. A tcgen05 GEMM with 128 x 256
+ * tiles, one head per column tile, whose epilogue writes the two halves of a
+ * tile straight into k_nope and v. All pointers 16-byte aligned; B, T as in
+ * mla_attn_prefill with B*T <= 2^31 - 129. Timeouts go to the device-wide
+ * word (mla_device_status).
+ */
+mla_status_t mla_kv_up_proj(const mla_bf16* c_kv, const mla_bf16* W_kv_b, int B, int T,
+                            mla_bf16* k_nope, mla_bf16* v, mla_stream_t stream);
+
+/*
+ * Workspace bytes of mla_attn_oproj_latent: mla_attn_oproj_workspace_bytes
+ * plus k_nope and v (B*64*T*128*2 each, rounded up to 256).
+ */
+size_t mla_attn_oproj_latent_workspace_bytes(int B, int T, int has_mask);
+
+/*
+ * The whole path from the latent: mla_kv_up_proj into the workspace, then
+ * mla_attn_oproj on its k_nope and v. Arguments as in mla_attn_oproj with
+ * c_kv [B, T, 512] and W_kv_b [16384, 512] in place of k_nope and v (same
+ * pointer checks), and workspace of mla_attn_oproj_latent_workspace_bytes.
+ */
+mla_status_t mla_attn_oproj_latent(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* c_kv, const mla_bf16* k_pe_shared,
+                                   const mla_bf16* W_kv_b, const mla_bf16* mask, int64_t mask_ld,
+                                   int B, int T, float softmax_scale, const mla_bf16* W_o,
+                                   void* workspace, size_t workspace_bytes, mla_bf16* out,
+                                   mla_stream_t stream);
+
 /* Largest B*T mla_attn_oproj_noalloc accepts (its fixed scratch holds the
  * merged attention output of this many tokens: 64 MiB). */
 #define MLA_NOALLOC_MAX_TOKENS 4096
@@ -394,7 +440,8 @@ mla_status_t mla_attn_oproj_fp8(const mla_bf16* q_nope, const mla_bf16* q_pe,
 /*
  * Outcome of the last call that used `workspace` (a workspace given to
  * mla_attn_prefill, mla_attn_oproj, mla_attn_oproj_varlen,
- * mla_attn_prefill_rope, mla_attn_oproj_rope or mla_attn_oproj_fp8; that call
+ * mla_attn_prefill_rope, mla_attn_oproj_rope, mla_attn_oproj_latent or
+ * mla_attn_oproj_fp8; that call
  * must have been enqueued on `stream` or be complete). Synchronises `stream`, then reads the call's status word.
  * Returns MLA_ERR_TIMEOUT if one of that call's kernels gave up on a bounded
  * wait, MLA_ERR_CUDA if the stream reports an error, MLA_ERR_INVALID_ARG for

@@ -79,6 +79,12 @@ _SIGNATURES = {
     "mla_attn_oproj_rope": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _ROPE_P, _VP,
                                            ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_float, _VP, _VP, ctypes.c_size_t, _VP, _VP]),
+    "mla_kv_up_proj": (ctypes.c_int, [_VP, _VP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP]),
+    "mla_attn_oproj_latent_workspace_bytes": (ctypes.c_size_t,
+                                              [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mla_attn_oproj_latent": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_float, _VP,
+                                             _VP, ctypes.c_size_t, _VP, _VP]),
     "mla_quantize_act_fp8": (ctypes.c_int, [_VP, ctypes.c_int64, _VP, _VP, _VP]),
     "mla_quantize_weight_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP]),
     "mla_o_proj_fp8": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP]),
@@ -376,6 +382,60 @@ def attn_oproj_rope(q_nope, q_pe, k_nope, k_pe, v, W_o, position_ids=None, rope=
                                  _ptr(W_o), _ptr(workspace), ws_bytes, _ptr(out),
                                  _stream_handle(stream))
     _check("mla_attn_oproj_rope", st)
+    return out
+
+
+KV_RANK = 512  # MLA_KV_RANK
+
+
+def kv_up_proj(c_kv, W_kv_b, k_nope=None, v=None, stream=None):
+    """k_nope, v [B, 64, T, 128] (bf16) from the latent c_kv [B, T, 512] and
+    W_kv_b [16384, 512] via ``mla_kv_up_proj``."""
+    lib = load()
+    B, T, _ = c_kv.shape
+    _req(c_kv, (B, T, KV_RANK), "c_kv")
+    _req(W_kv_b, (H * (DN + DV), KV_RANK), "W_kv_b")
+    if k_nope is None:
+        k_nope = torch.empty((B, H, T, DN), dtype=torch.bfloat16, device=c_kv.device)
+    if v is None:
+        v = torch.empty((B, H, T, DV), dtype=torch.bfloat16, device=c_kv.device)
+    _req(k_nope, (B, H, T, DN), "k_nope")
+    _req(v, (B, H, T, DV), "v")
+    st = lib.mla_kv_up_proj(_ptr(c_kv), _ptr(W_kv_b), B, T, _ptr(k_nope), _ptr(v),
+                            _stream_handle(stream))
+    _check("mla_kv_up_proj", st)
+    return k_nope, v
+
+
+def attn_oproj_latent_workspace_bytes(B: int, T: int, has_mask: bool) -> int:
+    return int(load().mla_attn_oproj_latent_workspace_bytes(B, T, int(bool(has_mask))))
+
+
+def attn_oproj_latent(q_nope, q_pe, c_kv, k_pe, W_kv_b, W_o, mask=None, softmax_scale=None,
+                      out=None, workspace=None, stream=None):
+    """Whole path from the latent (up-projection, attention, o_proj),
+    [B, T, 7168] bf16, via ``mla_attn_oproj_latent``."""
+    lib = load()
+    B, _, T, _ = q_nope.shape
+    _req(q_nope, (B, H, T, DN), "q_nope")
+    _req(q_pe, (B, H, T, DR), "q_pe")
+    _req(c_kv, (B, T, KV_RANK), "c_kv")
+    _req(k_pe, (B, 1, T, DR), "k_pe")
+    _req(W_kv_b, (H * (DN + DV), KV_RANK), "W_kv_b")
+    _req(W_o, (D_MODEL, K_OPROJ), "W_o")
+    mask_ld = _mask_ld(mask, B, T)
+    scale = _inputs.DEFAULT_SCALE if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty((B, T, D_MODEL), dtype=torch.bfloat16, device=q_nope.device)
+    _req(out, (B, T, D_MODEL), "out")
+    if workspace is None:
+        workspace = torch.empty(attn_oproj_latent_workspace_bytes(B, T, mask is not None),
+                                dtype=torch.uint8, device=q_nope.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib.mla_attn_oproj_latent(_ptr(q_nope), _ptr(q_pe), _ptr(c_kv), _ptr(k_pe),
+                                   _ptr(W_kv_b), _ptr(mask), mask_ld, B, T, scale, _ptr(W_o),
+                                   _ptr(workspace), ws_bytes, _ptr(out), _stream_handle(stream))
+    _check("mla_attn_oproj_latent", st)
     return out
 
 

@@ -364,6 +364,67 @@ mla_status_t mla_attn_oproj_rope(const mla_bf16* q_nope, const mla_bf16* q_pe,
                                      device_sm_count(), wait_limit_ns(), 0, err, st));
 }
 
+mla_status_t mla_kv_up_proj(const mla_bf16* c_kv, const mla_bf16* W_kv_b, int B, int T,
+                            mla_bf16* k_nope, mla_bf16* v, mla_stream_t stream) {
+  CallRange range("mla_kv_up_proj");
+  if (!c_kv || !W_kv_b || !k_nope || !v) return MLA_ERR_INVALID_ARG;
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT || int64_t(B) * int64_t(T) > kMaxM)
+    return MLA_ERR_SHAPE;
+  if (!aligned16(c_kv) || !aligned16(W_kv_b) || !aligned16(k_nope) || !aligned16(v))
+    return MLA_ERR_MISALIGNED;
+  mla_status_t s = check_device();
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_kv_up(c_kv, W_kv_b, k_nope, v, B, T, MLA_KV_RANK, device_sm_count(),
+                                wait_limit_ns(), device_error_word(),
+                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_attn_oproj_latent_workspace_bytes(int B, int T, int has_mask) {
+  if (B < 1 || T < 1 || B > kMaxB || T > kMaxT) return 0;
+  // status | k_nope | v | merged attention | mask classes
+  const size_t kv = round_up(size_t(B) * MLA_NUM_HEADS * size_t(T) * MLA_QK_NOPE_DIM * 2, 256);
+  return mla_attn_oproj_workspace_bytes(B, T, has_mask) + 2 * kv;
+}
+
+mla_status_t mla_attn_oproj_latent(const mla_bf16* q_nope, const mla_bf16* q_pe,
+                                   const mla_bf16* c_kv, const mla_bf16* k_pe_shared,
+                                   const mla_bf16* W_kv_b, const mla_bf16* mask, int64_t mask_ld,
+                                   int B, int T, float softmax_scale, const mla_bf16* W_o,
+                                   void* workspace, size_t workspace_bytes, mla_bf16* out,
+                                   mla_stream_t stream) {
+  CallRange range("mla_attn_oproj_latent");
+  // the up-projection's outputs stand in for k_nope and v in the checks
+  mla_status_t s = check_attn_args(q_nope, q_pe, c_kv, k_pe_shared, W_kv_b, mask, mask_ld, B, T,
+                                   softmax_scale, out);
+  if (s != MLA_OK) return s;
+  if (!W_o) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(W_o)) return MLA_ERR_MISALIGNED;
+  if (int64_t(B) * int64_t(T) > kMaxM) return MLA_ERR_SHAPE;
+  const size_t need = mla_attn_oproj_latent_workspace_bytes(B, T, mask != nullptr);
+  if (!workspace || workspace_bytes < need) return MLA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return MLA_ERR_MISALIGNED;
+  s = check_device();
+  if (s != MLA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int* err = call_status_word(workspace, st, &s);
+  if (s != MLA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace) + MLA_WORKSPACE_STATUS_BYTES;
+  const size_t kv = round_up(size_t(B) * MLA_NUM_HEADS * size_t(T) * MLA_QK_NOPE_DIM * 2, 256);
+  const size_t attn_bytes = round_up(size_t(B) * size_t(T) * MLA_OPROJ_IN * 2, 256);
+  uint8_t* k_nope = ws;
+  uint8_t* v = ws + kv;
+  uint8_t* attn = ws + 2 * kv;
+  void* cls = mask ? attn + attn_bytes : nullptr;
+  s = from_cuda(launch_kv_up(c_kv, W_kv_b, k_nope, v, B, T, MLA_KV_RANK, device_sm_count(),
+                             wait_limit_ns(), err, st));
+  if (s != MLA_OK) return s;
+  s = run_attention(q_nope, q_pe, k_nope, k_pe_shared, v, mask, mask_ld, B, T, softmax_scale,
+                    cls, attn, st, err);
+  if (s != MLA_OK) return s;
+  return from_cuda(launch_oproj_gemm(attn, W_o, out, int64_t(B) * T, MLA_HIDDEN, MLA_OPROJ_IN,
+                                     device_sm_count(), wait_limit_ns(), 0, err, st));
+}
+
 mla_status_t mla_quantize_act_fp8(const mla_bf16* x, int64_t M, uint8_t* q, float* scale,
                                   mla_stream_t stream) {
   CallRange range("mla_quantize_act_fp8");

@@ -66,13 +66,18 @@ struct GemmCfg {
                 "TMEM columns must be a power of two in [32, 512]");
 };
 
-template <int BN, int STAGES, int MT>
+// kSplit (the latent up-projection): the 256 columns of column tile nb are
+// head nb's 128 non-rotary key parts and 128 values; row m is token
+// (m / T, m % T). They are stored into C = k_nope [B, 64, T, 128] and
+// C2 = v [B, 64, T, 128] instead of a row-major [M, N] C.
+template <int BN, int STAGES, int MT, bool kSplit = false>
 __global__ void __launch_bounds__(kThreads, 1)
     oproj_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmB, __nv_bfloat16* __restrict__ C,
                       int M, int N, int K, unsigned long long wait_limit_ns,
-                      unsigned int* err_word) {
+                      unsigned int* err_word, __nv_bfloat16* __restrict__ C2, int T) {
   using Cfg = GemmCfg<BN, STAGES, MT>;
+  static_assert(!kSplit || (BN == 256 && MT == 1), "head split: one head per 256-wide tile");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t full_bar[STAGES];
   __shared__ uint64_t empty_bar[STAGES];
@@ -232,6 +237,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < MT; ++t) {
       const int row = mb * kTileM + t * kBM + row_in_tile;
       __nv_bfloat16* crow = C + size_t(row) * size_t(N) + size_t(nb) * BN;
+      __nv_bfloat16* vrow = nullptr;
+      if constexpr (kSplit) {
+        const int bi = row / T;  // row = bi * T + ti
+        const size_t off =
+            ((size_t(bi) * size_t(N / BN) + nb) * size_t(T) + (row - bi * T)) * (BN / 2);
+        crow = C + off;
+        vrow = C2 + off;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -244,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
         if (row < M) {
           uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+          if constexpr (kSplit)  // chunks 0..3: key part, 4..7: value
+            dst = reinterpret_cast<uint4*>((c < 4 ? crow : vrow) + (c & 3) * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
@@ -283,7 +298,39 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const void* W, __nv_bfloat16* C, i
   const int num_tiles = m_tiles * (N / BN);
   const int grid = num_tiles < num_sms ? num_tiles : num_sms;
   kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(tmA, tmB, C, M, N, K, wait_limit_ns,
-                                                   err_word);
+                                                   err_word, nullptr, 0);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- latent up-projection
+cudaError_t launch_kv_up_impl(const void* c_kv, const void* W, void* k_nope, void* v, int B, int T,
+                              int R, int num_sms, unsigned long long wait_limit_ns,
+                              unsigned int* err_word, cudaStream_t stream) {
+  constexpr int BN = 256, STAGES = 4;
+  using Cfg = GemmCfg<BN, STAGES, 1>;
+  const int64_t M64 = int64_t(B) * T;
+  const int N = 64 * BN;
+  if (M64 <= 0 || M64 > (int64_t(1) << 31) - kBM || R % kBK != 0) return cudaErrorInvalidValue;
+  const int M = int(M64);
+  CUtensorMap tmA, tmB;
+  const uint64_t a_dims[2] = {uint64_t(R), uint64_t(M)};
+  const uint64_t w_dims[2] = {uint64_t(R), uint64_t(N)};
+  const uint64_t strides[1] = {uint64_t(R) * 2};
+  const uint32_t a_box[2] = {kBK, kBM};
+  const uint32_t w_box[2] = {kBK, BN};
+  if (!encode_tmap_bf16(&tmA, c_kv, 2, a_dims, strides, a_box, true) ||
+      !encode_tmap_bf16(&tmB, W, 2, w_dims, strides, w_box, true))
+    return cudaErrorInvalidValue;
+  auto kern = oproj_gemm_kernel<BN, STAGES, 1, true>;
+  static ContextCache attr_done;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(Cfg::kSmemBytes),
+                                   &attr_done);
+  if (e != cudaSuccess) return e;
+  const int num_tiles = ((M + kBM - 1) / kBM) * (N / BN);
+  const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+  kern<<<grid, kThreads, Cfg::kSmemBytes, stream>>>(
+      tmA, tmB, static_cast<__nv_bfloat16*>(k_nope), M, N, R, wait_limit_ns, err_word,
+      static_cast<__nv_bfloat16*>(v), T);
   return cudaGetLastError();
 }
 
@@ -524,6 +571,12 @@ cudaError_t launch_small_m(const void* A, const void* W, __nv_bfloat16* C, int M
 }
 
 }  // namespace
+
+cudaError_t launch_kv_up(const void* c_kv, const void* W, void* k_nope, void* v, int B, int T,
+                         int R, int num_sms, unsigned long long wait_limit_ns,
+                         unsigned int* err_word, cudaStream_t stream) {
+  return launch_kv_up_impl(c_kv, W, k_nope, v, B, T, R, num_sms, wait_limit_ns, err_word, stream);
+}
 
 OprojTile oproj_pick_tile(int64_t M, int N, int num_sms) {
   // Largest expected throughput: fraction of the last wave's SMs kept busy,

@@ -18,6 +18,14 @@ cudaError_t launch_oproj_gemm(const void* A, const void* W, void* C, int64_t M, 
                               int num_sms, unsigned long long wait_limit_ns, int force_bn,
                               unsigned int* err_word, cudaStream_t stream, int test_stall = 0);
 
+// Up-projection of the compressed KV latent: kv = c_kv [B*T, R] . W [64*256, R]^T,
+// stored per head as k_nope [B, 64, T, 128] (columns h*256 .. +127) and
+// v [B, 64, T, 128] (columns h*256+128 .. +255), bf16, fp32 accumulation. The
+// tiled GEMM with 128 x 256 tiles (one head per column tile); R % 64 == 0.
+cudaError_t launch_kv_up(const void* c_kv, const void* W, void* k_nope, void* v, int B, int T,
+                         int R, int num_sms, unsigned long long wait_limit_ns,
+                         unsigned int* err_word, cudaStream_t stream);
+
 // Output tile the launcher picks for an M x N problem (M > 128) on `num_sms`
 // SMs: mt row blocks of 128 by bn columns.
 struct OprojTile {

@@ -254,3 +254,21 @@ def test_rope_argument_errors(lib):
     assert rope_call(lib, ws=A + 8) == MISALIGNED
     assert lib.mla_attn_oproj_rope(A, A, A, A, A, None, ctypes.byref(binding._yarn(None)), None,
                                    0, 1, 64, 0.07, None, A, 1 << 40, A, None) == INVALID
+
+
+def test_latent_workspace_sizes_and_argument_errors(lib):
+    kv = 64 * 64 * 128 * 2  # k_nope or v of B=1, T=64
+    assert lib.mla_attn_oproj_latent_workspace_bytes(1, 64, 0) == ST + 64 * 8192 * 2 + 2 * kv
+    assert lib.mla_attn_oproj_latent_workspace_bytes(0, 64, 0) == 0
+    up = lib.mla_kv_up_proj
+    assert up(None, A, 1, 64, A, A, None) == INVALID
+    assert up(A, A, 1, 64, A, None, None) == INVALID
+    assert up(A, A, 0, 64, A, A, None) == SHAPE
+    assert up(A, A, 1, 0, A, A, None) == SHAPE
+    assert up(A + 2, A, 1, 64, A, A, None) == MISALIGNED
+    assert up(A, A, 1, 64, A + 8, A, None) == MISALIGNED
+    lat = lib.mla_attn_oproj_latent
+    assert lat(A, A, None, A, A, None, 0, 1, 64, 0.07, A, A, 1 << 40, A, None) == INVALID
+    assert lat(A, A, A, A, A, None, 0, 1, 64, 0.07, None, A, 1 << 40, A, None) == INVALID
+    assert lat(A, A, A, A, A, None, 0, 1, 64, 0.07, A, A, ST + 64 * 8192 * 2, A, None) == WORKSPACE
+    assert lat(A, A, A, A, A + 2, None, 0, 1, 64, 0.07, A, A, 1 << 40, A, None) == MISALIGNED
