@@ -408,6 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
     tmem_alloc(&tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  __syncwarp();
   tc_fence_before();
   // Both CTAs' barriers are initialised before either can touch the other's.
   cluster_sync();
@@ -537,6 +538,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kSmallThreads, 1)
   // partial or arriving on its part_done). After a timeout on either side
   // those accesses can still come late, so both CTAs meet here first. Every
   // wait above is bounded, so every thread of both CTAs reaches this barrier.
+  __syncwarp();  // the .aligned cluster barrier wants converged warps
   tc_fence_before();
   cluster_sync();
   if (warp == 1) {
