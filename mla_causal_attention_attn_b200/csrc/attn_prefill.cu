@@ -43,6 +43,7 @@
 #include "attn_prefill.h"
 
 #include <cstdlib>
+#include <cstring>
 
 #include "host_util.h"
 #include "sm100.cuh"
@@ -831,9 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
-// The causal / valid-length kernel on a pair of SMs. A cluster of two CTAs
-// computes query tiles 2p (even CTA) and 2p+1 (odd CTA) of one (b, h); each
-// SM holds one 128-row query tile, and each score and PV product is ONE
+// The attention kernel on a pair of SMs. A cluster of two CTAs computes query
+// tiles 2p (even CTA) and 2p+1 (odd CTA) of one (b, h): each SM holds one
+// 128-row query tile, and each score and PV product is ONE
 // tcgen05.mma.cta_group::2 of M = 256 rows issued by the even CTA:
 //   S (256 x 128 keys, K = 128 nope + 64 rope): each CTA holds its 128 query
 //     rows and 64 of the 128 keys (the B operand is split by columns);
@@ -845,11 +846,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // the softmax of tile j runs. Issue order of the even CTA's MMA thread:
 //   S_0, S_1, [P_0] PV_0, S_2, [P_1] PV_1, S_3, ...
 // (P_j aliases S_j's buffer; S_{j+2} reuses it after PV_j in issue order).
+//
+// A cluster works on two items, query-tile pairs p and n_pairs - 1 - p of the
+// same (b, h) (one item for the middle pair when n_pairs is odd), so every
+// cluster visits the same number of key tiles, and one launch, barrier set
+// and tensor-memory allocation serve both. Both items' query tiles are loaded
+// up front (two query buffers) and each item accumulates into its own O, so
+// the key-tile sequence runs on across the item boundary: the second item's
+// first scores are computed while the first item's last softmax runs.
 // Roles (256 threads):
-//   warp 0       TMA producer of this CTA: its query tile, then per visited
-//                key tile its halves: k_nope lo / hi and k_pe of 64 keys, and
-//                V of all 128 keys for its 64 value dims (five 8 KB blocks)
-//                into a 20-block ring; each copy signals this CTA's barrier;
+//   warp 0       TMA producer of this CTA: its two query tiles, then per
+//                visited key tile its halves: k_nope lo / hi and k_pe of 64
+//                keys, and V of all 128 keys for its 64 value dims (five 8 KB
+//                blocks) into a 15-block ring; each copy signals this CTA's
+//                own barrier;
 //   warp 1       tensor-memory allocation for the pair; in the even CTA, the
 //                MMA-issuing thread;
 //   warp 2       odd CTA only: relays "query tile / ring block landed" to the
@@ -858,20 +868,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                before it leaves);
 //   warp 3       idle;
 //   warps 4..7   softmax of this CTA's 128 rows (one row per thread) and the
-//                epilogue O / l -> bf16 -> out.
-// Tensor memory (512 columns, allocated for the pair): S buffers at columns
-// 0 and 128, O at 256. Both CTAs meet at a cluster barrier before either
-// releases tensor memory or leaves.
+//                epilogue O / l -> bf16 -> out of each item.
+// Tensor memory (512 columns, allocated for the pair): S buffers at columns 0
+// and 128, O of item i at 256 + 128 i. Both CTAs meet at a cluster barrier
+// before either releases tensor memory or leaves.
 constexpr int kThreadsPair = 256;
 constexpr uint32_t kHalfBlock = 64 * 64 * 2;  // 64 rows x 64 bf16, 128-byte swizzle: 8 KB
-constexpr int kRingPair = 20;                  // 8 KB blocks: four key tiles
+constexpr int kRingPair = 15;                  // 8 KB blocks: three key tiles
 constexpr int kBlocksPerTilePair = 5;
-constexpr uint32_t kOffRingPair = kQBytes;     // after this CTA's query tile (48 KB)
+constexpr uint32_t kOffRingPair = 2 * kQBytes;  // after the two query tiles (96 KB)
 constexpr uint32_t kSmemPairUsed = kOffRingPair + kRingPair * kHalfBlock;
 constexpr size_t kSmemPairBytes = kSmemPairUsed + 1024;
-constexpr uint32_t kColOPair = 256;
+constexpr uint32_t kColOPair = 256;  // O of item i at kColOPair + 128 i
 constexpr uint16_t kPairMask = 0x3;  // both CTAs of the cluster
 static_assert(kSmemPairBytes <= 227 * 1024, "shared memory budget");
+
+// The items of a cluster and the tiles each visits.
+template <bool kMasked>
+struct PairItems {
+  int n_items;
+  int pair[2];
+  PairTiles<kMasked> tiles[2];
+  int n_visit[2];
+  __device__ __forceinline__ int total() const { return n_visit[0] + (n_items > 1 ? n_visit[1] : 0); }
+};
 
 template <bool kMasked, bool kRope>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
@@ -881,15 +901,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
                                  const __grid_constant__ CUtensorMap tmKp,
                                  const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ uint64_t q_full;      // this CTA's query tile landed
-  __shared__ uint64_t q_rot;       // its rotary part is rotated (4 softmax warps)
-  __shared__ uint64_t q_peer;      // even CTA: the odd CTA's query tile is ready
+  __shared__ uint64_t q_full[2];   // this CTA's query tile of item i landed
+  __shared__ uint64_t q_rot[2];    // its rotary part is rotated (4 softmax warps)
+  __shared__ uint64_t q_peer[2];   // even CTA: the odd CTA's query tile of item i is ready
   __shared__ uint64_t ring_full[kRingPair], ring_empty[kRingPair];
   __shared__ uint64_t peer_full[kRingPair];  // even CTA: the odd CTA's block landed
   __shared__ uint64_t s_full[2];   // S buffer b holds the next scores
   __shared__ uint64_t p_full[2];   // even CTA: P in buffer b written by all 8 softmax warps
   __shared__ uint64_t pv_done;     // one phase per PV product
-  __shared__ uint64_t o_final;
+  __shared__ uint64_t o_final[2];  // item i's last PV product has landed
   __shared__ uint64_t drain_bar;
   __shared__ uint64_t never_bar;   // no thread ever arrives (failure-detection test)
   __shared__ uint32_t tmem_slot;
@@ -903,51 +923,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
-  // cluster -> (b, h, pair): groups of kHeadGroup heads, longest pairs first
+  // cluster -> (b, h, item pair): groups of kHeadGroup heads; within a group
+  // the clusters of the longest item first
+  const int n_cl = (args.n_pairs + 1) / 2;  // clusters per (b, h)
   const int cid = int(blockIdx.x >> 1);
-  const int per_group = kHeadGroup * args.n_pairs;
+  const int per_group = kHeadGroup * n_cl;
   const int grp = cid / per_group;
   const int rem = cid - grp * per_group;
   const int b = grp / (kH / kHeadGroup);
   const int h = (grp % (kH / kHeadGroup)) * kHeadGroup + rem % kHeadGroup;
-  const int pair = args.n_pairs - 1 - rem / kHeadGroup;
+  const int ci = rem / kHeadGroup;
   const int bh = b * kH + h;
   const int n_keys =
       (!kMasked && args.valid_len) ? min(max(args.valid_len[b], 0), args.T) : args.T;
 
-  PairTiles<kMasked> tiles;
+  PairItems<kMasked> items;
+  items.pair[0] = args.n_pairs - 1 - ci;
+  items.pair[1] = ci;
+  items.n_items = items.pair[1] < items.pair[0] ? 2 : 1;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    tiles.qt[i] = 2 * pair + i;
-    tiles.exists[i] = tiles.qt[i] < args.n_qt;
-    tiles.cls[i] = (kMasked && args.tile_class && tiles.exists[i])
-                       ? args.tile_class + (size_t(b) * args.n_qt + tiles.qt[i]) * args.n_kv
-                       : nullptr;
+  for (int it = 0; it < 2; ++it) {
+    PairTiles<kMasked>& t = items.tiles[it];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      t.qt[i] = 2 * items.pair[it] + i;
+      t.exists[i] = it < items.n_items && t.qt[i] < args.n_qt;
+      t.cls[i] = (kMasked && args.tile_class && t.exists[i])
+                     ? args.tile_class + (size_t(b) * args.n_qt + t.qt[i]) * args.n_kv
+                     : nullptr;
+    }
+    t.kv_end = (n_keys + kBKV - 1) / kBKV;
+    t.end = kMasked ? args.n_kv : min(min(2 * items.pair[it] + 2, args.n_qt), t.kv_end);
+    int nv = 0;
+    if (it < items.n_items)
+      for (int kt = t.first(); kt < t.end; kt = t.next(kt)) ++nv;
+    items.n_visit[it] = nv;
   }
-  tiles.kv_end = (n_keys + kBKV - 1) / kBKV;
-  tiles.end = kMasked ? args.n_kv : min(min(2 * pair + 2, args.n_qt), tiles.kv_end);
-  int n_visit = 0;
-  for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) ++n_visit;
-  const int qt_me = tiles.qt[rank];
+  const int n_total = items.total();
 
   WaitCtl ctl{&abort_flag, args.wait_limit_ns, kErrKernelAttn, args.err_word};
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(&q_full, 1);
-    mbar_init(&q_rot, 4);
-    mbar_init(&q_peer, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_rot[i], 4);
+      mbar_init(&q_peer[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 8);
+      mbar_init(&o_final[i], 1);
+    }
     for (int s = 0; s < kRingPair; ++s) {
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
       mbar_init(&peer_full[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);
-    }
     mbar_init(&pv_done, 1);
-    mbar_init(&o_final, 1);
     mbar_init(&drain_bar, 1);
     mbar_init(&never_bar, 1);
     fence_barrier_init();
@@ -964,20 +995,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_visit > 0) {
+    if (lane == 0 && n_total > 0) {
       prefetch_tensormap(&tmQn);
       prefetch_tensormap(&tmQp);
       prefetch_tensormap(&tmKn);
       prefetch_tensormap(&tmKp);
       prefetch_tensormap(&tmV);
-      const int q0 = qt_me * kBQ;
-      mbar_arrive_expect_tx(&q_full, kQBytes);
-      tma_load_3d(smem, &tmQn, &q_full, 0, q0, bh);
-      tma_load_3d(smem + kBlock, &tmQn, &q_full, 64, q0, bh);
-      tma_load_3d(smem + 2 * kBlock, &tmQp, &q_full, 0, q0, bh);
+      uint32_t q_issued = 0;
+      for (int it = 0; it < items.n_items; ++it) {
+        if (items.n_visit[it] == 0) continue;
+        const int q0 = items.tiles[it].qt[rank] * kBQ;
+        uint8_t* sQ = smem + it * kQBytes;
+        mbar_arrive_expect_tx(&q_full[it], kQBytes);
+        tma_load_3d(sQ, &tmQn, &q_full[it], 0, q0, bh);
+        tma_load_3d(sQ + kBlock, &tmQn, &q_full[it], 64, q0, bh);
+        tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full[it], 0, q0, bh);
+        q_issued |= 1u << it;
+      }
       const int kh = int(rank) * 64;  // this CTA's keys of a tile / its value dims
       auto prefetch_tile = [&](int pt) {
-        if (pt >= tiles.end) return;
         const int p0 = pt * kBKV;
         tma_prefetch_l2_3d(&tmKn, 0, p0 + kh, bh);
         tma_prefetch_l2_3d(&tmKn, 64, p0 + kh, bh);
@@ -985,54 +1021,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         tma_prefetch_l2_3d(&tmV, kh, p0, bh);
         tma_prefetch_l2_3d(&tmV, kh, p0 + 64, bh);
       };
-      int pf = tiles.next(tiles.first());
-      prefetch_tile(pf);
       uint32_t issued = 0, issued_par = 0;
       uint32_t s = 0;
       bool ok = true;
-      for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt)) {
-        const int k0 = kt * kBKV;
-        if (pf < tiles.end) {
-          pf = tiles.next(pf);
-          prefetch_tile(pf);
-        }
-#pragma unroll 1
-        for (int i = 0; i < kBlocksPerTilePair; ++i, ++s) {
-          const uint32_t slot = s % kRingPair;
-          const uint32_t par = (s / kRingPair) & 1u;
-          if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
-          uint8_t* dst = smem + kOffRingPair + slot * kHalfBlock;
-          mbar_arrive_expect_tx(&ring_full[slot], kHalfBlock);
-          switch (i) {
-            case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0 + kh, bh); break;
-            case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0 + kh, bh); break;
-            case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0 + kh, b); break;
-            default: tma_load_3d(dst, &tmV, &ring_full[slot], kh, k0 + (i - 3) * 64, bh); break;
+      for (int it = 0; ok && it < items.n_items; ++it) {
+        const PairTiles<kMasked>& t = items.tiles[it];
+        int pf = t.next(t.first());
+        if (pf < t.end) prefetch_tile(pf);
+        for (int kt = t.first(); ok && kt < t.end; kt = t.next(kt)) {
+          const int k0 = kt * kBKV;
+          if (pf < t.end) {
+            pf = t.next(pf);
+            if (pf < t.end) prefetch_tile(pf);
           }
-          issued |= 1u << slot;
-          issued_par = (issued_par & ~(1u << slot)) | (par << slot);
+#pragma unroll 1
+          for (int i = 0; i < kBlocksPerTilePair; ++i, ++s) {
+            const uint32_t slot = s % kRingPair;
+            const uint32_t par = (s / kRingPair) & 1u;
+            if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
+            uint8_t* dst = smem + kOffRingPair + slot * kHalfBlock;
+            mbar_arrive_expect_tx(&ring_full[slot], kHalfBlock);
+            switch (i) {
+              case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0 + kh, bh); break;
+              case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0 + kh, bh); break;
+              case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0 + kh, b); break;
+              default: tma_load_3d(dst, &tmV, &ring_full[slot], kh, k0 + (i - 3) * 64, bh); break;
+            }
+            issued |= 1u << slot;
+            issued_par = (issued_par & ~(1u << slot)) | (par << slot);
+          }
         }
       }
       if (!ok) {
         // let the copies already issued land before the CTA's memory goes away
         int zero = 0;
         WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
-        mbar_wait(&q_full, 0, drain, 2);
+        for (int it = 0; it < 2; ++it)
+          if (q_issued & (1u << it)) mbar_wait(&q_full[it], 0, drain, 2);
         for (int k = 0; k < kRingPair; ++k)
           if (issued & (1u << k)) mbar_wait(&ring_full[k], (issued_par >> k) & 1u, drain, 3);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (lane == 0 && leader && n_visit > 0) {
+    if (lane == 0 && leader && n_total > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(2 * kBQ, kBKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(2 * kBQ, kDV, false, true);
       const uint32_t ring0 = smem_u32(smem + kOffRingPair);
-      const uint32_t sQ = smem_u32(smem);
-      const uint32_t o_tmem = tmem_base + kColOPair;
-      bool ok = mbar_wait(&q_full, 0, ctl, 10) && mbar_wait_cluster_sleep(&q_peer, 0, ctl, 10);
-      if (kRope && ok) ok = mbar_wait(&q_rot, 0, ctl, 16);
+      const int n0 = items.n_visit[0];  // the first item's tiles come first
+      bool ok = true;
       bool issued_any = false;
+      uint32_t q_ready = 0;
       auto block_addr = [&](uint32_t seq) { return ring0 + (seq % kRingPair) * kHalfBlock; };
       // a block of both CTAs has landed
       auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
@@ -1040,12 +1079,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         return mbar_wait(&ring_full[slot], par, ctl, site) &&
                mbar_wait_cluster_sleep(&peer_full[slot], par, ctl, site);
       };
-      auto release = [&](uint32_t seq) { mma_commit_pair_mc(&ring_empty[seq % kRingPair], kPairMask); };
+      auto release = [&](uint32_t seq) {
+        mma_commit_pair_mc(&ring_empty[seq % kRingPair], kPairMask);
+      };
       auto issue_s = [&](int j) -> bool {
+        const int it = j < n0 ? 0 : 1;
+        if (!(q_ready & (1u << it))) {
+          // both CTAs' query tiles of this item are in shared memory (rotated)
+          if (!mbar_wait(&q_full[it], 0, ctl, 10) ||
+              !mbar_wait_cluster_sleep(&q_peer[it], 0, ctl, 10))
+            return false;
+          if (kRope && !mbar_wait(&q_rot[it], 0, ctl, 16)) return false;
+          q_ready |= 1u << it;
+        }
         const uint32_t base = uint32_t(j) * kBlocksPerTilePair;
         if (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13))
           return false;
         tc_fence_after();
+        const uint32_t sQ = smem_u32(smem + it * kQBytes);
         const uint32_t s_tmem = tmem_base + 128u * uint32_t(j & 1);
 #pragma unroll
         for (int blk = 0; blk < 3; ++blk) {
@@ -1063,32 +1114,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         release(base + 2);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && n_visit > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n_visit; ++j) {
+      ok = issue_s(0);
+      if (ok && n_total > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n_total; ++j) {
+        const int it = j < n0 ? 0 : 1;
+        const int first = it == 0 ? 0 : n0;  // the item's first tile overwrites its O
         const uint32_t base = uint32_t(j) * kBlocksPerTilePair;
-        if (!mbar_wait_cluster_sleep(&p_full[j & 1], uint32_t(j >> 1) & 1u, ctl, 11)) { ok = false; break; }
+        if (!mbar_wait_cluster_sleep(&p_full[j & 1], uint32_t(j >> 1) & 1u, ctl, 11)) {
+          ok = false;
+          break;
+        }
         if (!wait_block(base + 3, 12) || !wait_block(base + 4, 12)) { ok = false; break; }
         tc_fence_after();
         // P_j: 128 keys as 64 packed columns of buffer j & 1; V: each CTA's
         // 64 value dims of 64 keys per block, MN-major, 8-key groups 1 KB apart.
         const uint32_t p_tmem = tmem_base + 128u * uint32_t(j & 1);
+        const uint32_t o_tmem = tmem_base + kColOPair + 128u * uint32_t(it);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const uint32_t vb = block_addr(base + 3 + half);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (j > 0 || half > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (j > first || half > 0 || kk > 0) ? 1u : 0u;
             const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kHalfBlock, 1024);
             mma_ts_pair(o_tmem, p_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
           }
         }
         mma_commit_pair_mc(&pv_done, kPairMask);
+        if (j == first + items.n_visit[it] - 1) mma_commit_pair_mc(&o_final[it], kPairMask);
         release(base + 3);
         release(base + 4);
-        if (j + 2 < n_visit && !issue_s(j + 2)) { ok = false; break; }
+        if (j + 2 < n_total && !issue_s(j + 2)) { ok = false; break; }
       }
-      if (ok) mma_commit_pair_mc(&o_final, kPairMask);
       if (!ok && issued_any) {
         mma_commit_pair_mc(&drain_bar, 0x1);
         int zero = 0;
@@ -1098,12 +1155,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ relay (odd CTA)
-    if (lane == 0 && !leader && n_visit > 0) {
-      const uint32_t q_peer_remote = mapa_shared(smem_u32(&q_peer), 0);
-      bool ok = mbar_wait(&q_full, 0, ctl, 17);
-      if (kRope && ok) ok = mbar_wait(&q_rot, 0, ctl, 17);
-      if (ok) mbar_arrive_cluster(q_peer_remote);
-      const uint32_t n_blocks = uint32_t(n_visit) * kBlocksPerTilePair;
+    if (lane == 0 && !leader && n_total > 0) {
+      bool ok = true;
+      for (int it = 0; ok && it < items.n_items; ++it) {
+        if (items.n_visit[it] == 0) continue;
+        ok = mbar_wait(&q_full[it], 0, ctl, 17);
+        if (kRope && ok) ok = mbar_wait(&q_rot[it], 0, ctl, 17);
+        if (ok) mbar_arrive_cluster(mapa_shared(smem_u32(&q_peer[it]), 0));
+      }
+      const uint32_t n_blocks = uint32_t(n_total) * kBlocksPerTilePair;
       for (uint32_t s = 0; ok && s < n_blocks; ++s) {
         const uint32_t slot = s % kRingPair;
         if (!mbar_wait(&ring_full[slot], (s / kRingPair) & 1u, ctl, 18)) { ok = false; break; }
@@ -1114,227 +1174,246 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
     // ------------------------------------------------------------ softmax / epilogue
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // row within the tile == TMEM lane
-    const int q = qt_me * kBQ + r;
     const uint32_t lane_base = tmem_addr(tmem_base, quad * 32, 0);
-    const bool row_valid = tiles.exists[rank] && q < args.T;
-    const __nv_bfloat16* mrow =
-        (kMasked && row_valid) ? args.mask + (size_t(b) * args.T + q) * args.mask_ld : nullptr;
     const uint32_t p_full_remote[2] = {mapa_shared(smem_u32(&p_full[0]), 0),
                                        mapa_shared(smem_u32(&p_full[1]), 0)};
     bool ok = true;
-    if (kRope && n_visit > 0) {
-      // rotate this row's q_pe in shared memory (see the one-SM kernel)
-      ok = mbar_wait(&q_full, 0, ctl, 24);
-      if (ok && row_valid) {
-        uint8_t* rowp = smem + 2 * kBlock + r * 128;
-        const float4* cs =
-            reinterpret_cast<const float4*>(args.rope_cs + (size_t(b) * args.T + q) * 32);
+    if (kRope) {
+      // rotate this row's q_pe in shared memory, for each item (see the
+      // one-SM kernel)
+      for (int it = 0; it < items.n_items; ++it) {
+        if (items.n_visit[it] == 0) continue;
+        const int q = items.tiles[it].qt[rank] * kBQ + r;
+        if (ok) ok = mbar_wait(&q_full[it], 0, ctl, 24);
+        if (ok && items.tiles[it].exists[rank] && q < args.T) {
+          uint8_t* rowp = smem + it * kQBytes + 2 * kBlock + r * 128;
+          const float4* cs =
+              reinterpret_cast<const float4*>(args.rope_cs + (size_t(b) * args.T + q) * 32);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* chunk = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
-          uint4 w = *chunk;
-          const float4 a = __ldg(cs + 2 * c), bq = __ldg(cs + 2 * c + 1);
-          const float csn[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+          for (int c = 0; c < 8; ++c) {
+            uint4* chunk = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
+            uint4 w = *chunk;
+            const float4 a = __ldg(cs + 2 * c), bq = __ldg(cs + 2 * c + 1);
+            const float csn[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = bf16_bits_to_float(wp[e] & 0xffffu);
-            const float x1 = bf16_bits_to_float(wp[e] >> 16);
-            const float cc = csn[2 * e], ss = csn[2 * e + 1];
-            wp[e] = pack_bf16x2(fmaf(x0, cc, -x1 * ss), fmaf(x1, cc, x0 * ss));
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = bf16_bits_to_float(wp[e] & 0xffffu);
+              const float x1 = bf16_bits_to_float(wp[e] >> 16);
+              const float cc = csn[2 * e], ss = csn[2 * e + 1];
+              wp[e] = pack_bf16x2(fmaf(x0, cc, -x1 * ss), fmaf(x1, cc, x0 * ss));
+            }
+            *chunk = w;
           }
-          *chunk = w;
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_rot[it]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&q_rot);
     }
 
-    float m = -INFINITY;  // running max, log2 units
-    float l = 0.f;        // running sum of p (fp32, unrounded)
-    uint32_t n = 0;       // key tiles used by this row's tile so far
-    int j = 0;            // visited key tiles so far (the pair's sequence)
-    for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt), ++j) {
-      const int buf = j & 1;
-      const uint32_t colS = 128u * uint32_t(buf);
-      const int k0 = kt * kBKV;
-      if (args.test_stall && rank == 0 && blockIdx.x == 0 &&
-          !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
+    int j = 0;  // visited key tiles so far (the pair's sequence, over both items)
+    for (int it = 0; it < items.n_items; ++it) {
+      const PairTiles<kMasked>& tiles = items.tiles[it];
+      const int qt_me = tiles.qt[rank];
+      const int q = qt_me * kBQ + r;
+      const bool row_valid = tiles.exists[rank] && q < args.T;
+      const __nv_bfloat16* mrow =
+          (kMasked && row_valid) ? args.mask + (size_t(b) * args.T + q) * args.mask_ld : nullptr;
+      float m = -INFINITY;  // running max, log2 units
+      float l = 0.f;        // running sum of p (fp32, unrounded)
+      uint32_t n = 0;       // key tiles used by this row's tile so far
+      for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt), ++j) {
+        const int buf = j & 1;
+        const uint32_t colS = 128u * uint32_t(buf);
+        const int k0 = kt * kBKV;
+        if (args.test_stall && rank == 0 && blockIdx.x == 0 &&
+            !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_warp(&s_full[buf], uint32_t(j >> 1) & 1u, ctl, 20)) { ok = false; break; }
+        tc_fence_after();
+        if (!tiles.active(int(rank), kt)) {
+          // No key of this tile is allowed for this CTA's rows (causal: the
+          // odd CTA's diagonal tile seen from the even CTA; a mask: a skipped
+          // tile): P = 0 for the pair's PV.
+          uint32_t z[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) z[i] = 0u;
+          tmem_st32(lane_base + colS, z);
+          tmem_st32(lane_base + colS + 32, z);
+        } else {
+          // as in the one-SM kernel: the fast route for tiles that need no
+          // mask entries added (every causal tile; all-zero, causal-pattern
+          // and prefix tiles of a mask) with a per-row key limit, the exact
+          // two-pass route for the others and for a non-positive scale
+          const uint8_t tile_cls = kMasked ? (tiles.cls[rank] ? tiles.cls[rank][kt]
+                                                              : uint8_t(kTileMixed))
+                                           : uint8_t(kTileZero);
+          ScoreChunk<kMasked> sc;
+          sc.cls = (kMasked && row_valid) ? tile_cls : uint8_t(kTileZero);
+          sc.row_valid = row_valid;
+          sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
+          sc.kvalid = args.T - k0;
+          sc.mask_vec = args.mask_vec;
+          const bool causal_tile = !kMasked ? kt == qt_me : tile_cls == kTileCausal;
+          const bool prefix_tile = kMasked && tile_cls >= kTilePrefix;
+          const bool fast_route =
+              (tile_cls == kTileZero || tile_cls == kTileCausal || prefix_tile) &&
+              args.scale_log2 > 0.f;
+          const int key_end = kMasked ? args.T : n_keys;
+          const bool diag = causal_tile || prefix_tile || key_end - k0 < kBKV;
+          const int lim =
+              min(causal_tile ? r : (prefix_tile ? int(tile_cls) - kTilePrefix : kBKV - 1),
+                  key_end - 1 - k0);
+          sc.diag_row = (kMasked ? (causal_tile || prefix_tile) : diag) ? lim : kBKV;
+          uint32_t raw[kBKV];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
+          tmem_ld_wait();
+          reg_fence(raw);
+          float alpha = 1.f;
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          bool exact = !(fast_route && n > 0);
+          float rowsum = 0.f;
+          if (!exact) {
+#pragma unroll
+            for (int c2 = 0; c2 < 4; c2 += 2) {
+              uint32_t pk[32];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
+                if (diag)
+                  p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, lim, args.scale_log2, m,
+                                       ph, acc);
+                else
+                  p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m,
+                                        ph, acc);
+              }
+              tmem_st32(lane_base + colS + 16 * c2, pk);
+            }
+            rowsum =
+                ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            if (__any_sync(0xffffffffu, !(rowsum <= 256.f))) {
+              const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
+                               args.scale_log2;
+              exact = __any_sync(0xffffffffu, !(mt <= m + kRescaleThreshold));
+              if (exact) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+              }
+            }
+          }
+          if (exact) {
+            float mt;
+            if (fast_route) {
+              mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
+              mt *= args.scale_log2;
+            } else {
+              float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                float x[32];
+                sc.apply(raw + c * 32, c, args.scale_log2, 0.f, x);
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                  m4[0] = fmax3(m4[0], x[i], x[i + 1]);
+                  m4[1] = fmax3(m4[1], x[i + 2], x[i + 3]);
+                  m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
+                  m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) raw[c * 32 + i] = __float_as_uint(x[i]);
+              }
+              mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            }
+            float m_new = m;
+            if (n == 0) {
+              m_new = mt;
+            } else if (mt > m + kRescaleThreshold) {
+              m_new = mt;
+              alpha = fast_exp2(m - m_new);
+            }
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            m = m_new;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint32_t* rc = raw + c * 32;
+              uint32_t pk[16];
+              if (fast_route) {
+                if (diag)
+                  p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
+                else
+                  p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
+              } else {
+                float x[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(rc[i]) - m_use;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float p0 = fast_exp2(x[2 * i]);
+                  const float p1 = fast_exp2(x[2 * i + 1]);
+                  fadd2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)],
+                        acc[2 * (i & 3) + 1], p0, p1);
+                  pk[i] = pack_bf16x2(p0, p1);
+                }
+              }
+              tmem_st16(lane_base + colS + 16 * c, pk);
+            }
+            rowsum =
+                ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            // Rescale this item's O once PV_{j-1} (the last product issued
+            // before this tile's, into the same O since n > 0) has landed;
+            // PV_j waits for this tile's P below.
+            if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+              if (!mbar_wait_warp(&pv_done, uint32_t(j - 1) & 1u, ctl, 21)) {
+                ok = false;
+              } else {
+                tc_fence_after();
+                const uint32_t colO = kColOPair + 128u * uint32_t(it);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                  uint32_t rr[32];
+                  tmem_ld32(lane_base + colO + c * 32, rr);
+                  tmem_ld_wait();
+                  reg_fence(rr);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i)
+                    rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+                  tmem_st32(lane_base + colO + c * 32, rr);
+                }
+              }
+            }
+          }  // exact
+          l = l * alpha + rowsum;
+          ++n;
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full_remote[buf]);
+      }
+      if (!ok) break;
+
+      // epilogue of this item: O / l -> bf16 -> out[b, q, h*128 + e]. Every
+      // softmax thread waits for the item's last product, so no MMA is in
+      // flight at teardown.
+      const bool have = items.n_visit[it] > 0 && mbar_wait_warp(&o_final[it], 0, ctl, 22);
+      if (items.n_visit[it] > 0 && !have) {
         ok = false;
         break;
       }
-      if (!mbar_wait_warp(&s_full[buf], uint32_t(j >> 1) & 1u, ctl, 20)) { ok = false; break; }
-      tc_fence_after();
-      if (!tiles.active(int(rank), kt)) {
-        // No key of this tile is allowed for this CTA's rows (causal: the
-        // odd CTA's diagonal tile seen from the even CTA; a mask: a skipped
-        // tile): P = 0 for the pair's PV.
-        uint32_t z[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0u;
-        tmem_st32(lane_base + colS, z);
-        tmem_st32(lane_base + colS + 32, z);
-      } else {
-        // as in the one-SM kernel: the fast route for tiles that need no
-        // mask entries added (every causal tile; all-zero, causal-pattern
-        // and prefix tiles of a mask) with a per-row key limit, the exact
-        // two-pass route for the others and for a non-positive scale
-        const uint8_t tile_cls = kMasked ? (tiles.cls[rank] ? tiles.cls[rank][kt]
-                                                            : uint8_t(kTileMixed))
-                                         : uint8_t(kTileZero);
-        ScoreChunk<kMasked> sc;
-        sc.cls = (kMasked && row_valid) ? tile_cls : uint8_t(kTileZero);
-        sc.row_valid = row_valid;
-        sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
-        sc.kvalid = args.T - k0;
-        sc.mask_vec = args.mask_vec;
-        const bool causal_tile = !kMasked ? kt == qt_me : tile_cls == kTileCausal;
-        const bool prefix_tile = kMasked && tile_cls >= kTilePrefix;
-        const bool fast_route =
-            (tile_cls == kTileZero || tile_cls == kTileCausal || prefix_tile) &&
-            args.scale_log2 > 0.f;
-        const int key_end = kMasked ? args.T : n_keys;
-        const bool diag = causal_tile || prefix_tile || key_end - k0 < kBKV;
-        const int lim = min(causal_tile ? r : (prefix_tile ? int(tile_cls) - kTilePrefix : kBKV - 1),
-                            key_end - 1 - k0);
-        sc.diag_row = (kMasked ? (causal_tile || prefix_tile) : diag) ? lim : kBKV;
-        uint32_t raw[kBKV];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
-        tmem_ld_wait();
-        reg_fence(raw);
-        float alpha = 1.f;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        bool exact = !(fast_route && n > 0);
-        float rowsum = 0.f;
-        if (!exact) {
-#pragma unroll
-          for (int c2 = 0; c2 < 4; c2 += 2) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
-              if (diag)
-                p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, lim, args.scale_log2, m, ph,
-                                     acc);
-              else
-                p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph,
-                                      acc);
-            }
-            tmem_st32(lane_base + colS + 16 * c2, pk);
-          }
-          rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-          if (__any_sync(0xffffffffu, !(rowsum <= 256.f))) {
-            const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
-                             args.scale_log2;
-            exact = __any_sync(0xffffffffu, !(mt <= m + kRescaleThreshold));
-            if (exact) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            }
-          }
-        }
-        if (exact) {
-          float mt;
-          if (fast_route) {
-            mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
-            mt *= args.scale_log2;
-          } else {
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float x[32];
-              sc.apply(raw + c * 32, c, args.scale_log2, 0.f, x);
-#pragma unroll
-              for (int i = 0; i < 32; i += 8) {
-                m4[0] = fmax3(m4[0], x[i], x[i + 1]);
-                m4[1] = fmax3(m4[1], x[i + 2], x[i + 3]);
-                m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
-                m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
-              }
-#pragma unroll
-              for (int i = 0; i < 32; ++i) raw[c * 32 + i] = __float_as_uint(x[i]);
-            }
-            mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          }
-          float m_new = m;
-          if (n == 0) {
-            m_new = mt;
-          } else if (mt > m + kRescaleThreshold) {
-            m_new = mt;
-            alpha = fast_exp2(m - m_new);
-          }
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          m = m_new;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t* rc = raw + c * 32;
-            uint32_t pk[16];
-            if (fast_route) {
-              if (diag)
-                p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
-              else
-                p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
-            } else {
-              float x[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(rc[i]) - m_use;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float p0 = fast_exp2(x[2 * i]);
-                const float p1 = fast_exp2(x[2 * i + 1]);
-                fadd2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)],
-                      acc[2 * (i & 3) + 1], p0, p1);
-                pk[i] = pack_bf16x2(p0, p1);
-              }
-            }
-            tmem_st16(lane_base + colS + 16 * c, pk);
-          }
-          rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-          // Rescale O once PV_{j-1} (the last product issued before this
-          // tile's) has landed; PV_j waits for this tile's P below.
-          if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-            if (j > 0 && !mbar_wait_warp(&pv_done, uint32_t(j - 1) & 1u, ctl, 21)) {
-              ok = false;
-            } else {
-              tc_fence_after();
-#pragma unroll 1
-              for (int c = 0; c < 4; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(lane_base + kColOPair + c * 32, rr);
-                tmem_ld_wait();
-                reg_fence(rr);
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-                tmem_st32(lane_base + kColOPair + c * 32, rr);
-              }
-            }
-          }
-        }  // exact
-        l = l * alpha + rowsum;
-        ++n;
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(p_full_remote[buf]);
-    }
-
-    // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]. Every softmax thread
-    // waits for the last product, so no MMA is in flight at teardown.
-    const bool have = ok && n_visit > 0 && mbar_wait_warp(&o_final, 0, ctl, 22);
-    if (have) tc_fence_after();
-    if (n == 0 || have) {
+      if (have) tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = args.out + (size_t(b) * args.T + q) * size_t(kH * kDV) + h * kDV;
+      const uint32_t colO = kColOPair + 128u * uint32_t(it);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
         if (n > 0) {
-          tmem_ld32(lane_base + kColOPair + c * 32, rr);
+          tmem_ld32(lane_base + colO + c * 32, rr);
           tmem_ld_wait();
           reg_fence(rr);
         } else {
@@ -1448,12 +1527,12 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// MLA_ATTN_ONE_SM=1 (read once; diagnostics and A/B timing) runs the causal and
-// valid-length calls on the one-SM kernel instead of the CTA-pair kernel.
-bool one_sm_kernel_forced() {
+// Which kernel runs the causal and valid-length calls: MLA_ATTN_KERNEL=pair
+// (read once) selects the CTA-pair kernel, anything else the one-SM kernel.
+bool pair_kernel_selected() {
   static const bool v = [] {
-    const char* s = std::getenv("MLA_ATTN_ONE_SM");
-    return s && s[0] == '1' && s[1] == '\0';
+    const char* s = std::getenv("MLA_ATTN_KERNEL");
+    return s && std::strcmp(s, "pair") == 0;
   }();
   return v;
 }
@@ -1499,7 +1578,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   if (mask && valid_len) return cudaErrorInvalidValue;
   CUtensorMap tmQn, tmQp, tmKn, tmKp, tmV;
   const int BH = B * kH;
-  if (!mask && !one_sm_kernel_forced()) {
+  if (!mask && pair_kernel_selected()) {
     // CTA pairs: K maps with 64-key boxes (each CTA loads half the keys)
     if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
         !make_map_3d(&tmKn, k_nope, kDN, T, BH, 64) || !make_map_3d(&tmKp, k_pe, kDR, T, B, 64) ||
@@ -1524,7 +1603,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
     a.err_word = err_word;
     a.test_stall = test_stall;
     a.rope_cs = static_cast<const float2*>(rope_cs);
-    const long long ctas = 2LL * B * kH * a.n_pairs;
+    const long long ctas = 2LL * B * kH * ((a.n_pairs + 1) / 2);  // a cluster per two items
     if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
     kern<<<unsigned(ctas), kThreadsPair, kSmemPairBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV,
                                                                   a);
