@@ -200,15 +200,6 @@ struct ScoreChunk {
   }
 };
 
-// Exponentials moved from the MUFU unit to the FMA pipe (exp2_poly2): pair i
-// of a chunk goes to the polynomial when kUseExp2Poly and (i & kPolyMask) ==
-// kPolyMask. Off: measured on B200 at B=1, T=4096, the softmax warps are bound
-// by issue slots and latency rather than MUFU throughput, and moving one pair
-// in four (or more) to the 10-instruction polynomial made the kernel slower
-// (0.400 ms without, 0.427 ms at 1/4, 0.464 ms at 1/2).
-constexpr bool kUseExp2Poly = false;
-constexpr int kPolyMask = 3;
-
 // Maximum of a row of 128 raw scores; on the diagonal tile keys c > r are
 // excluded (causal).
 template <bool kDiag>
@@ -230,12 +221,11 @@ __device__ __forceinline__ float raw_row_max(const uint32_t (&raw)[kBKV], int r)
   return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 }
 
-// Causal tile, 32 raw scores of chunk c: p = 2^(s*scale_log2 - m), packed as
-// bf16 pairs into pk and summed (unrounded, fp32) into the paired partial sums
-// acc. On the diagonal tile keys c > r give 0, and every exponential goes to
-// MUFU (which maps -inf to exactly 0); elsewhere the FMA-pipe polynomial may
-// take some pairs (kUseExp2Poly). With kTrackMax, xmax[0..1] also collect the
-// largest s*scale_log2 - m seen (the caller's running-max check).
+// Causal tile, 32 raw scores of chunk c: p = 2^(s*scale_log2 - m) (MUFU
+// ex2, which maps -inf to exactly 0), packed as bf16 pairs into pk and summed
+// (unrounded, fp32) into the paired partial sums acc. On the diagonal tile
+// keys c > r give 0. With kTrackMax, xmax[0..1] also collect the largest
+// s*scale_log2 - m seen (the caller's running-max check).
 template <bool kDiag, bool kTrackMax = false>
 __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r, float scale_log2,
                                                float m, uint32_t (&pk)[16], float (&acc)[8],
@@ -251,15 +241,8 @@ __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r
       if (c * 32 + 2 * i + 1 > r) x1 = -INFINITY;
     }
     if (kTrackMax) xmax[i & 1] = fmax3(xmax[i & 1], x0, x1);
-    if (kDiag) {
-      p0 = fast_exp2(x0);
-      p1 = fast_exp2(x1);
-    } else if (kUseExp2Poly && (i & kPolyMask) == kPolyMask) {
-      exp2_poly2(x0, x1, p0, p1);
-    } else {
-      p0 = fast_exp2(x0);
-      p1 = fast_exp2(x1);
-    }
+    p0 = fast_exp2(x0);
+    p1 = fast_exp2(x1);
     const int a = 2 * (i & 3);
     fadd2(acc[a], acc[a + 1], acc[a], acc[a + 1], p0, p1);
     pk[i] = pack_bf16x2(p0, p1);

@@ -615,29 +615,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two values on the FMA pipe (no MUFU), for x >= -125 after a clamp
-// (smaller x give ~2^-125, not 0; callers use it only where that is fine).
-// Cody-Waite range reduction: n = round(x) via the 1.5*2^23 rounding
-// constant, f = x - n in [-1/2, 1/2], 2^f from a cubic minimax polynomial
-// (coefficients from fit_exp2_poly.py, max relative error 8.4e-5), and the
-// result's exponent field raised by n.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& e0, float& e1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.999919593334198f, c1 = 0.6932621598243713f,
-                  c2 = 0.24271419644355774f, c3 = 0.055213067680597305f;
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  float t0, t1, n0, n1, f0, f1, p0, p1;
-  fadd2(t0, t1, x0, x1, kRound, kRound);    // low mantissa bits of t hold round(x)
-  fadd2(n0, n1, t0, t1, -kRound, -kRound);  // n = round(x), exact
-  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
-  ffma2(p0, p1, c3, c3, f0, f1, c2, c2);
-  ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
-  ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
-  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
