@@ -825,44 +825,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 //     memory, each CTA holds 64 of the 128 value dims of all 128 keys.
 // So every K/V byte a CTA loads serves 256 query rows, as in the one-SM
 // kernel, while each SM runs a single softmax warpgroup (its 128 rows), and
-// S is double-buffered in tensor memory: S of key tile j+1 is computed while
-// the softmax of tile j runs. Issue order of the even CTA's MMA thread:
-//   S_0, S_1, [P_0] PV_0, S_2, [P_1] PV_1, S_3, ...
-// (P_j aliases S_j's buffer; S_{j+2} reuses it after PV_j in issue order).
+// S is triple-buffered in tensor memory: the scores of the next two key tiles
+// are computed or queued while the softmax of one tile runs. Issue order of
+// the even CTA's MMA thread:
+//   S_0, S_1, S_2, [P_0] PV_0, S_3, [P_1] PV_1, S_4, ...
+// (P_j aliases S_j's buffer; S_{j+3} reuses it after PV_j in issue order).
 //
 // A cluster works on two items, query-tile pairs p and n_pairs - 1 - p of the
 // same (b, h) (one item for the middle pair when n_pairs is odd), so every
-// cluster visits the same number of key tiles, and one launch, barrier set
-// and tensor-memory allocation serve both. Both items' query tiles are loaded
-// up front (two query buffers) and each item accumulates into its own O, so
-// the key-tile sequence runs on across the item boundary: the second item's
-// first scores are computed while the first item's last softmax runs.
+// cluster visits the same number of key tiles and one launch, barrier set and
+// tensor-memory allocation serve both. Both items' query tiles are loaded up
+// front (two query buffers); the key-tile sequence runs on across the item
+// boundary, and the items share one O accumulator (the second item's first
+// PV, which overwrites O, waits for its first P, which the softmax threads
+// write only after they have read the first item's O).
+//
+// Cross-CTA signals, chosen for their cost on B200 (a remote mbarrier arrive
+// with release at cluster scope stalls its thread for about 0.7 us, so no
+// per-block or per-softmax-warp thread handshake crosses the pair):
+//  - ring blocks: both CTAs' TMA copies complete on the even CTA's barrier
+//    (cp.async.bulk.tensor .cta_group::2); the even CTA arms both CTAs' bytes;
+//  - query tiles: each CTA's copies complete on its own barrier (the odd
+//    CTA's softmax warps rotate them under the rotary calls), and a helper
+//    thread of the odd CTA forwards "ready" once per item;
+//  - P: the softmax warps arrive on a barrier of their own CTA; the odd CTA's
+//    helper forwards its CTA's P once per key tile.
 // Roles (256 threads):
 //   warp 0       TMA producer of this CTA: its two query tiles, then per
 //                visited key tile its halves: k_nope lo / hi and k_pe of 64
 //                keys, and V of all 128 keys for its 64 value dims (five 8 KB
-//                blocks) into a 15-block ring; each copy signals this CTA's
-//                own barrier;
+//                blocks) into a 15-block ring;
 //   warp 1       tensor-memory allocation for the pair; in the even CTA, the
 //                MMA-issuing thread;
-//   warp 2       odd CTA only: relays "query tile / ring block landed" to the
-//                even CTA with remote mbarrier arrivals (no copy ever signals
-//                the other CTA's barrier, so each CTA can drain its own copies
-//                before it leaves);
+//   warp 2       odd CTA only: the helper forwarding query and P readiness;
 //   warp 3       idle;
 //   warps 4..7   softmax of this CTA's 128 rows (one row per thread) and the
 //                epilogue O / l -> bf16 -> out of each item.
-// Tensor memory (512 columns, allocated for the pair): S buffers at columns 0
-// and 128, O of item i at 256 + 128 i. Both CTAs meet at a cluster barrier
-// before either releases tensor memory or leaves.
+// Tensor memory (512 columns, allocated for the pair): S buffers at columns
+// 0, 128 and 256, O at 384.
+//
+// Teardown: after a first cluster barrier no CTA issues another copy; the
+// even CTA then makes the last phase of every ring slot complete (arming, or
+// completing with mbarrier.complete_tx, the bytes of a copy that only one of
+// the two CTAs issued before an abort) and waits for it, so no copy is in
+// flight toward either CTA; a second cluster barrier precedes the release of
+// tensor memory and the exit.
 constexpr int kThreadsPair = 256;
 constexpr uint32_t kHalfBlock = 64 * 64 * 2;  // 64 rows x 64 bf16, 128-byte swizzle: 8 KB
 constexpr int kRingPair = 15;                  // 8 KB blocks: three key tiles
 constexpr int kBlocksPerTilePair = 5;
+constexpr int kSBufs = 3;                      // score buffers in tensor memory
 constexpr uint32_t kOffRingPair = 2 * kQBytes;  // after the two query tiles (96 KB)
 constexpr uint32_t kSmemPairUsed = kOffRingPair + kRingPair * kHalfBlock;
 constexpr size_t kSmemPairBytes = kSmemPairUsed + 1024;
-constexpr uint32_t kColOPair = 256;  // O of item i at kColOPair + 128 i
+constexpr uint32_t kColOPair = 384;
 constexpr uint16_t kPairMask = 0x3;  // both CTAs of the cluster
 static_assert(kSmemPairBytes <= 227 * 1024, "shared memory budget");
 
@@ -887,14 +903,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   __shared__ uint64_t q_full[2];   // this CTA's query tile of item i landed
   __shared__ uint64_t q_rot[2];    // its rotary part is rotated (4 softmax warps)
   __shared__ uint64_t q_peer[2];   // even CTA: the odd CTA's query tile of item i is ready
-  __shared__ uint64_t ring_full[kRingPair], ring_empty[kRingPair];
-  __shared__ uint64_t peer_full[kRingPair];  // even CTA: the odd CTA's block landed
-  __shared__ uint64_t s_full[2];   // S buffer b holds the next scores
-  __shared__ uint64_t p_full[2];   // even CTA: P in buffer b written by all 8 softmax warps
-  __shared__ uint64_t pv_done;     // one phase per PV product
-  __shared__ uint64_t o_final[2];  // item i's last PV product has landed
+  __shared__ uint64_t ring_full[kRingPair];   // even CTA: both CTAs' halves of a block landed
+  __shared__ uint64_t ring_empty[kRingPair];  // this CTA's slot is free again
+  __shared__ uint64_t s_full[kSBufs];  // S buffer b holds the next scores
+  __shared__ uint64_t p_full[kSBufs];  // even CTA: P in buffer b is complete (4 warps + helper);
+                                       // odd CTA: its 4 softmax warps wrote their P
+  __shared__ uint64_t pv_done[kSBufs];  // PV of the tile whose P was in buffer b landed
+                                        // (per buffer: a waiter is never two phases behind)
+  __shared__ uint64_t o_final;     // one phase per item: its last PV product has landed
   __shared__ uint64_t drain_bar;
   __shared__ uint64_t never_bar;   // no thread ever arrives (failure-detection test)
+  __shared__ uint32_t n_issued;    // ring blocks this CTA's producer issued
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -948,20 +967,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
+    n_issued = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_rot[i], 4);
       mbar_init(&q_peer[i], 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);
-      mbar_init(&o_final[i], 1);
+      mbar_init(&p_full[i], leader ? 5 : 4);
+      mbar_init(&pv_done[i], 1);
     }
     for (int s = 0; s < kRingPair; ++s) {
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_empty[s], 1);
-      mbar_init(&peer_full[s], 1);
     }
-    mbar_init(&pv_done, 1);
+    mbar_init(&o_final, 1);
     mbar_init(&drain_bar, 1);
     mbar_init(&never_bar, 1);
     fence_barrier_init();
@@ -972,7 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   }
   __syncwarp();  // the .aligned cluster barrier wants converged warps
   tc_fence_before();
-  cluster_sync();  // both CTAs' barriers initialised before any remote arrival
+  cluster_sync();  // both CTAs' barriers initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
@@ -1004,7 +1025,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         tma_prefetch_l2_3d(&tmV, kh, p0, bh);
         tma_prefetch_l2_3d(&tmV, kh, p0 + 64, bh);
       };
-      uint32_t issued = 0, issued_par = 0;
       uint32_t s = 0;
       bool ok = true;
       for (int it = 0; ok && it < items.n_items; ++it) {
@@ -1023,27 +1043,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
             const uint32_t par = (s / kRingPair) & 1u;
             if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
             uint8_t* dst = smem + kOffRingPair + slot * kHalfBlock;
-            mbar_arrive_expect_tx(&ring_full[slot], kHalfBlock);
+            // both CTAs' copies of this block complete on the even CTA's barrier
+            if (leader) mbar_arrive_expect_tx(&ring_full[slot], 2 * kHalfBlock);
+            const uint32_t fb = mapa_shared(smem_u32(&ring_full[slot]), 0);
             switch (i) {
-              case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0 + kh, bh); break;
-              case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0 + kh, bh); break;
-              case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0 + kh, b); break;
-              default: tma_load_3d(dst, &tmV, &ring_full[slot], kh, k0 + (i - 3) * 64, bh); break;
+              case 0: tma_load_3d_pair(dst, &tmKn, fb, 0, k0 + kh, bh); break;
+              case 1: tma_load_3d_pair(dst, &tmKn, fb, 64, k0 + kh, bh); break;
+              case 2: tma_load_3d_pair(dst, &tmKp, fb, 0, k0 + kh, b); break;
+              default: tma_load_3d_pair(dst, &tmV, fb, kh, k0 + (i - 3) * 64, bh); break;
             }
-            issued |= 1u << slot;
-            issued_par = (issued_par & ~(1u << slot)) | (par << slot);
+            n_issued = s + 1;
           }
         }
       }
-      if (!ok) {
-        // let the copies already issued land before the CTA's memory goes away
-        int zero = 0;
-        WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
+      // the query copies complete on this CTA's own barriers: drain them here
+      int zero = 0;
+      WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
+      if (!ok)
         for (int it = 0; it < 2; ++it)
           if (q_issued & (1u << it)) mbar_wait(&q_full[it], 0, drain, 2);
-        for (int k = 0; k < kRingPair; ++k)
-          if (issued & (1u << k)) mbar_wait(&ring_full[k], (issued_par >> k) & 1u, drain, 3);
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
@@ -1051,16 +1069,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(2 * kBQ, kBKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(2 * kBQ, kDV, false, true);
       const uint32_t ring0 = smem_u32(smem + kOffRingPair);
+      const uint32_t o_tmem = tmem_base + kColOPair;
       const int n0 = items.n_visit[0];  // the first item's tiles come first
       bool ok = true;
       bool issued_any = false;
       uint32_t q_ready = 0;
       auto block_addr = [&](uint32_t seq) { return ring0 + (seq % kRingPair) * kHalfBlock; };
-      // a block of both CTAs has landed
       auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
-        const uint32_t slot = seq % kRingPair, par = (seq / kRingPair) & 1u;
-        return mbar_wait(&ring_full[slot], par, ctl, site) &&
-               mbar_wait_cluster_sleep(&peer_full[slot], par, ctl, site);
+        return mbar_wait(&ring_full[seq % kRingPair], (seq / kRingPair) & 1u, ctl, site);
       };
       auto release = [&](uint32_t seq) {
         mma_commit_pair_mc(&ring_empty[seq % kRingPair], kPairMask);
@@ -1080,7 +1096,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
           return false;
         tc_fence_after();
         const uint32_t sQ = smem_u32(smem + it * kQBytes);
-        const uint32_t s_tmem = tmem_base + 128u * uint32_t(j & 1);
+        const uint32_t s_tmem = tmem_base + 128u * uint32_t(j % kSBufs);
 #pragma unroll
         for (int blk = 0; blk < 3; ++blk) {
 #pragma unroll
@@ -1091,28 +1107,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
           }
         }
         issued_any = true;
-        mma_commit_pair_mc(&s_full[j & 1], kPairMask);
+        mma_commit_pair_mc(&s_full[j % kSBufs], kPairMask);
         release(base);
         release(base + 1);
         release(base + 2);
         return true;
       };
-      ok = issue_s(0);
-      if (ok && n_total > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < min(n_total, kSBufs); ++j) ok = issue_s(j);
       for (int j = 0; ok && j < n_total; ++j) {
         const int it = j < n0 ? 0 : 1;
-        const int first = it == 0 ? 0 : n0;  // the item's first tile overwrites its O
+        const int first = it == 0 ? 0 : n0;  // the item's first tile overwrites O
         const uint32_t base = uint32_t(j) * kBlocksPerTilePair;
-        if (!mbar_wait_cluster_sleep(&p_full[j & 1], uint32_t(j >> 1) & 1u, ctl, 11)) {
+        // (acquire at cluster scope: the odd CTA's P is forwarded by a remote arrive)
+        if (!mbar_wait_cluster_sleep(&p_full[j % kSBufs], uint32_t(j / kSBufs) & 1u, ctl, 11) ||
+            !wait_block(base + 3, 12) || !wait_block(base + 4, 12)) {
           ok = false;
           break;
         }
-        if (!wait_block(base + 3, 12) || !wait_block(base + 4, 12)) { ok = false; break; }
         tc_fence_after();
-        // P_j: 128 keys as 64 packed columns of buffer j & 1; V: each CTA's
-        // 64 value dims of 64 keys per block, MN-major, 8-key groups 1 KB apart.
-        const uint32_t p_tmem = tmem_base + 128u * uint32_t(j & 1);
-        const uint32_t o_tmem = tmem_base + kColOPair + 128u * uint32_t(it);
+        // P_j: 128 keys as 64 packed columns of its S buffer; V: each CTA's 64
+        // value dims of 64 keys per block, MN-major, 8-key groups 1 KB apart.
+        const uint32_t p_tmem = tmem_base + 128u * uint32_t(j % kSBufs);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const uint32_t vb = block_addr(base + 3 + half);
@@ -1123,11 +1138,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
             mma_ts_pair(o_tmem, p_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
           }
         }
-        mma_commit_pair_mc(&pv_done, kPairMask);
-        if (j == first + items.n_visit[it] - 1) mma_commit_pair_mc(&o_final[it], kPairMask);
+        mma_commit_pair_mc(&pv_done[j % kSBufs], kPairMask);
+        if (j == first + items.n_visit[it] - 1) mma_commit_pair_mc(&o_final, kPairMask);
         release(base + 3);
         release(base + 4);
-        if (j + 2 < n_total && !issue_s(j + 2)) { ok = false; break; }
+        if (j + kSBufs < n_total && !issue_s(j + kSBufs)) { ok = false; break; }
       }
       if (!ok && issued_any) {
         mma_commit_pair_mc(&drain_bar, 0x1);
@@ -1137,7 +1152,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ relay (odd CTA)
+    // ------------------------------------------------------------ helper (odd CTA)
     if (lane == 0 && !leader && n_total > 0) {
       bool ok = true;
       for (int it = 0; ok && it < items.n_items; ++it) {
@@ -1146,11 +1161,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         if (kRope && ok) ok = mbar_wait(&q_rot[it], 0, ctl, 17);
         if (ok) mbar_arrive_cluster(mapa_shared(smem_u32(&q_peer[it]), 0));
       }
-      const uint32_t n_blocks = uint32_t(n_total) * kBlocksPerTilePair;
-      for (uint32_t s = 0; ok && s < n_blocks; ++s) {
-        const uint32_t slot = s % kRingPair;
-        if (!mbar_wait(&ring_full[slot], (s / kRingPair) & 1u, ctl, 18)) { ok = false; break; }
-        mbar_arrive_cluster(mapa_shared(smem_u32(&peer_full[slot]), 0));
+      for (int j = 0; ok && j < n_total; ++j) {
+        if (!mbar_wait(&p_full[j % kSBufs], uint32_t(j / kSBufs) & 1u, ctl, 18)) break;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&p_full[j % kSBufs]), 0));
       }
     }
   } else if (warp >= 4) {
@@ -1158,8 +1171,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_base = tmem_addr(tmem_base, quad * 32, 0);
-    const uint32_t p_full_remote[2] = {mapa_shared(smem_u32(&p_full[0]), 0),
-                                       mapa_shared(smem_u32(&p_full[1]), 0)};
     bool ok = true;
     if (kRope) {
       // rotate this row's q_pe in shared memory, for each item (see the
@@ -1207,7 +1218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
       float l = 0.f;        // running sum of p (fp32, unrounded)
       uint32_t n = 0;       // key tiles used by this row's tile so far
       for (int kt = tiles.first(); ok && kt < tiles.end; kt = tiles.next(kt), ++j) {
-        const int buf = j & 1;
+        const int buf = j % kSBufs;
         const uint32_t colS = 128u * uint32_t(buf);
         const int k0 = kt * kBKV;
         if (args.test_stall && rank == 0 && blockIdx.x == 0 &&
@@ -1215,7 +1226,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
           ok = false;
           break;
         }
-        if (!mbar_wait_warp(&s_full[buf], uint32_t(j >> 1) & 1u, ctl, 20)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[buf], uint32_t(j / kSBufs) & 1u, ctl, 20)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (!tiles.active(int(rank), kt)) {
           // No key of this tile is allowed for this CTA's rows (causal: the
@@ -1347,25 +1361,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
             }
             rowsum =
                 ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-            // Rescale this item's O once PV_{j-1} (the last product issued
-            // before this tile's, into the same O since n > 0) has landed;
-            // PV_j waits for this tile's P below.
+            // Rescale O once PV_{j-1} (the last product issued before this
+            // tile's, into this item's O since n > 0) has landed; PV_j waits
+            // for this tile's P below.
             if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              if (!mbar_wait_warp(&pv_done, uint32_t(j - 1) & 1u, ctl, 21)) {
+              if (!mbar_wait_warp(&pv_done[(j - 1) % kSBufs], uint32_t((j - 1) / kSBufs) & 1u,
+                                  ctl, 21)) {
                 ok = false;
               } else {
                 tc_fence_after();
-                const uint32_t colO = kColOPair + 128u * uint32_t(it);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                   uint32_t rr[32];
-                  tmem_ld32(lane_base + colO + c * 32, rr);
+                  tmem_ld32(lane_base + kColOPair + c * 32, rr);
                   tmem_ld_wait();
                   reg_fence(rr);
 #pragma unroll
                   for (int i = 0; i < 32; ++i)
                     rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-                  tmem_st32(lane_base + colO + c * 32, rr);
+                  tmem_st32(lane_base + kColOPair + c * 32, rr);
                 }
               }
             }
@@ -1376,14 +1390,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(p_full_remote[buf]);
+        if (lane == 0) mbar_arrive(&p_full[buf]);  // own CTA; the helper forwards the odd CTA's
       }
       if (!ok) break;
 
       // epilogue of this item: O / l -> bf16 -> out[b, q, h*128 + e]. Every
-      // softmax thread waits for the item's last product, so no MMA is in
-      // flight at teardown.
-      const bool have = items.n_visit[it] > 0 && mbar_wait_warp(&o_final[it], 0, ctl, 22);
+      // softmax thread waits for the item's last product (so no MMA is in
+      // flight at teardown) and reads O before it writes the next item's
+      // first P (whose PV overwrites O).
+      const bool have = items.n_visit[it] > 0 && mbar_wait_warp(&o_final, uint32_t(it) & 1u, ctl, 22);
       if (items.n_visit[it] > 0 && !have) {
         ok = false;
         break;
@@ -1391,12 +1406,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
       if (have) tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       __nv_bfloat16* orow = args.out + (size_t(b) * args.T + q) * size_t(kH * kDV) + h * kDV;
-      const uint32_t colO = kColOPair + 128u * uint32_t(it);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
         if (n > 0) {
-          tmem_ld32(lane_base + colO + c * 32, rr);
+          tmem_ld32(lane_base + kColOPair + c * 32, rr);
           tmem_ld_wait();
           reg_fence(rr);
         } else {
@@ -1416,13 +1430,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
                                 packed[4 * i + 3]);
         }
       }
+      tc_fence_before();
     }
   }
 
-  // Neither CTA leaves, nor frees the pair's tensor memory, while the other
-  // may still arrive on its barriers or its MMAs read this CTA's memory.
+  // Teardown, first barrier: from here on neither CTA issues a copy.
   __syncwarp();
   tc_fence_before();
+  cluster_sync();
+  if (leader && warp == 0 && lane == 0 && n_total > 0) {
+    // Every ring copy completes on this CTA's barriers. Account for a block
+    // that only one CTA issued (possible only after an abort), then wait for
+    // the last phase of every slot; each slot has at most one phase pending.
+    const uint32_t n_own = n_issued;
+    const uint32_t n_peer = ld_shared_cluster_u32(mapa_shared(smem_u32(&n_issued), 1));
+    const uint32_t lo = min(n_own, n_peer), hi = max(n_own, n_peer);
+    for (uint32_t seq = lo; seq < hi; ++seq) {
+      uint64_t* fb = &ring_full[seq % kRingPair];
+      if (seq < n_own)  // armed for both CTAs' bytes, the odd CTA's copy never came
+        mbar_complete_tx_cluster(mapa_shared(smem_u32(fb), 0), kHalfBlock);
+      else              // the odd CTA's copy came, this CTA never armed the phase
+        mbar_arrive_expect_tx(fb, kHalfBlock);
+    }
+    int zero = 0;
+    WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
+    const uint32_t first = hi > uint32_t(kRingPair) ? hi - kRingPair : 0;
+    for (uint32_t seq = first; seq < hi; ++seq)
+      mbar_wait(&ring_full[seq % kRingPair], (seq / kRingPair) & 1u, drain, 3);
+  }
+  // Second barrier: no copy is in flight toward either CTA; neither leaves,
+  // nor frees the pair's tensor memory, before both get here.
+  __syncwarp();
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
