@@ -851,32 +851,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 //  - P: the softmax warps arrive on a barrier of their own CTA; the odd CTA's
 //    helper forwards its CTA's P once per key tile.
 // Roles (256 threads):
-//   warp 0       TMA producer of this CTA: its two query tiles, then per
-//                visited key tile its halves: k_nope lo / hi and k_pe of 64
-//                keys, and V of all 128 keys for its 64 value dims (five 8 KB
-//                blocks) into a 15-block ring;
+//   warp 0       K producer of this CTA: its two query tiles, then per
+//                visited key tile its halves of k_nope lo / hi and k_pe (64
+//                keys; three 8 KB blocks) into a 9-block ring;
 //   warp 1       tensor-memory allocation for the pair; in the even CTA, the
 //                MMA-issuing thread;
 //   warp 2       odd CTA only: the helper forwarding query and P readiness;
-//   warp 3       idle;
+//   warp 3       V producer: per visited key tile V of all 128 keys for this
+//                CTA's 64 value dims (two 8 KB blocks) into a 6-block ring.
+//                K and V have rings and producers of their own because their
+//                slots free up at different times (a K block after its S
+//                product, a V block only after its PV product, a softmax
+//                later): one ring filled in order would hold the K blocks of
+//                tile j+3 behind the V blocks of tile j+2, and so behind
+//                PV_{j-1};
 //   warps 4..7   softmax of this CTA's 128 rows (one row per thread) and the
 //                epilogue O / l -> bf16 -> out of each item.
 // Tensor memory (512 columns, allocated for the pair): S buffers at columns
 // 0, 128 and 256, O at 384.
 //
 // Teardown: after a first cluster barrier no CTA issues another copy; the
-// even CTA then makes the last phase of every ring slot complete (arming, or
+// even CTA then makes the last phase of every slot of both rings complete (arming, or
 // completing with mbarrier.complete_tx, the bytes of a copy that only one of
 // the two CTAs issued before an abort) and waits for it, so no copy is in
 // flight toward either CTA; a second cluster barrier precedes the release of
 // tensor memory and the exit.
 constexpr int kThreadsPair = 256;
 constexpr uint32_t kHalfBlock = 64 * 64 * 2;  // 64 rows x 64 bf16, 128-byte swizzle: 8 KB
-constexpr int kRingPair = 15;                  // 8 KB blocks: three key tiles
-constexpr int kBlocksPerTilePair = 5;
+constexpr int kKRing = 9;                      // K blocks: three key tiles
+constexpr int kVRing = 6;                      // V blocks: three key tiles
+constexpr int kKPerTile = 3, kVPerTile = 2;
 constexpr int kSBufs = 3;                      // score buffers in tensor memory
-constexpr uint32_t kOffRingPair = 2 * kQBytes;  // after the two query tiles (96 KB)
-constexpr uint32_t kSmemPairUsed = kOffRingPair + kRingPair * kHalfBlock;
+constexpr uint32_t kOffKRing = 2 * kQBytes;    // after the two query tiles (96 KB)
+constexpr uint32_t kOffVRing = kOffKRing + kKRing * kHalfBlock;
+constexpr uint32_t kSmemPairUsed = kOffVRing + kVRing * kHalfBlock;
 constexpr size_t kSmemPairBytes = kSmemPairUsed + 1024;
 constexpr uint32_t kColOPair = 384;
 constexpr uint16_t kPairMask = 0x3;  // both CTAs of the cluster
@@ -903,8 +911,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   __shared__ uint64_t q_full[2];   // this CTA's query tile of item i landed
   __shared__ uint64_t q_rot[2];    // its rotary part is rotated (4 softmax warps)
   __shared__ uint64_t q_peer[2];   // even CTA: the odd CTA's query tile of item i is ready
-  __shared__ uint64_t ring_full[kRingPair];   // even CTA: both CTAs' halves of a block landed
-  __shared__ uint64_t ring_empty[kRingPair];  // this CTA's slot is free again
+  __shared__ uint64_t k_full[kKRing];   // even CTA: both CTAs' halves of a K block landed
+  __shared__ uint64_t k_empty[kKRing];  // this CTA's K slot is free again
+  __shared__ uint64_t v_full[kVRing];   // even CTA: both CTAs' halves of a V block landed
+  __shared__ uint64_t v_empty[kVRing];
   __shared__ uint64_t s_full[kSBufs];  // S buffer b holds the next scores
   __shared__ uint64_t p_full[kSBufs];  // even CTA: P in buffer b is complete (4 warps + helper);
                                        // odd CTA: its 4 softmax warps wrote their P
@@ -913,7 +923,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   __shared__ uint64_t o_final;     // one phase per item: its last PV product has landed
   __shared__ uint64_t drain_bar;
   __shared__ uint64_t never_bar;   // no thread ever arrives (failure-detection test)
-  __shared__ uint32_t n_issued;    // ring blocks this CTA's producer issued
+  __shared__ uint32_t n_issued[2];  // K and V blocks this CTA's producers issued
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
@@ -967,7 +977,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    n_issued = 0;
+    n_issued[0] = 0;
+    n_issued[1] = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_rot[i], 4);
@@ -978,9 +989,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
       mbar_init(&p_full[i], leader ? 5 : 4);
       mbar_init(&pv_done[i], 1);
     }
-    for (int s = 0; s < kRingPair; ++s) {
-      mbar_init(&ring_full[s], 1);
-      mbar_init(&ring_empty[s], 1);
+    for (int s = 0; s < kKRing; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVRing; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(&o_final, 1);
     mbar_init(&drain_bar, 1);
@@ -997,33 +1012,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: the query tiles and the K blocks; warp 3: the V blocks
     if (lane == 0 && n_total > 0) {
-      prefetch_tensormap(&tmQn);
-      prefetch_tensormap(&tmQp);
-      prefetch_tensormap(&tmKn);
-      prefetch_tensormap(&tmKp);
-      prefetch_tensormap(&tmV);
+      const bool kprod = warp == 0;
       uint32_t q_issued = 0;
-      for (int it = 0; it < items.n_items; ++it) {
-        if (items.n_visit[it] == 0) continue;
-        const int q0 = items.tiles[it].qt[rank] * kBQ;
-        uint8_t* sQ = smem + it * kQBytes;
-        mbar_arrive_expect_tx(&q_full[it], kQBytes);
-        tma_load_3d(sQ, &tmQn, &q_full[it], 0, q0, bh);
-        tma_load_3d(sQ + kBlock, &tmQn, &q_full[it], 64, q0, bh);
-        tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full[it], 0, q0, bh);
-        q_issued |= 1u << it;
+      if (kprod) {
+        prefetch_tensormap(&tmQn);
+        prefetch_tensormap(&tmQp);
+        prefetch_tensormap(&tmKn);
+        prefetch_tensormap(&tmKp);
+        for (int it = 0; it < items.n_items; ++it) {
+          if (items.n_visit[it] == 0) continue;
+          const int q0 = items.tiles[it].qt[rank] * kBQ;
+          uint8_t* sQ = smem + it * kQBytes;
+          mbar_arrive_expect_tx(&q_full[it], kQBytes);
+          tma_load_3d(sQ, &tmQn, &q_full[it], 0, q0, bh);
+          tma_load_3d(sQ + kBlock, &tmQn, &q_full[it], 64, q0, bh);
+          tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full[it], 0, q0, bh);
+          q_issued |= 1u << it;
+        }
+      } else {
+        prefetch_tensormap(&tmV);
       }
       const int kh = int(rank) * 64;  // this CTA's keys of a tile / its value dims
+      const int per_tile = kprod ? kKPerTile : kVPerTile;
+      const uint32_t ring = kprod ? kKRing : kVRing;
+      uint64_t* full = kprod ? k_full : v_full;
+      uint64_t* empty = kprod ? k_empty : v_empty;
+      uint8_t* ring0 = smem + (kprod ? kOffKRing : kOffVRing);
       auto prefetch_tile = [&](int pt) {
         const int p0 = pt * kBKV;
-        tma_prefetch_l2_3d(&tmKn, 0, p0 + kh, bh);
-        tma_prefetch_l2_3d(&tmKn, 64, p0 + kh, bh);
-        tma_prefetch_l2_3d(&tmKp, 0, p0 + kh, b);
-        tma_prefetch_l2_3d(&tmV, kh, p0, bh);
-        tma_prefetch_l2_3d(&tmV, kh, p0 + 64, bh);
+        if (kprod) {
+          tma_prefetch_l2_3d(&tmKn, 0, p0 + kh, bh);
+          tma_prefetch_l2_3d(&tmKn, 64, p0 + kh, bh);
+          tma_prefetch_l2_3d(&tmKp, 0, p0 + kh, b);
+        } else {
+          tma_prefetch_l2_3d(&tmV, kh, p0, bh);
+          tma_prefetch_l2_3d(&tmV, kh, p0 + 64, bh);
+        }
       };
       uint32_t s = 0;
       bool ok = true;
@@ -1038,21 +1066,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
             if (pf < t.end) prefetch_tile(pf);
           }
 #pragma unroll 1
-          for (int i = 0; i < kBlocksPerTilePair; ++i, ++s) {
-            const uint32_t slot = s % kRingPair;
-            const uint32_t par = (s / kRingPair) & 1u;
-            if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
-            uint8_t* dst = smem + kOffRingPair + slot * kHalfBlock;
+          for (int i = 0; i < per_tile; ++i, ++s) {
+            const uint32_t slot = s % ring;
+            const uint32_t par = (s / ring) & 1u;
+            if (!mbar_wait(&empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
+            uint8_t* dst = ring0 + slot * kHalfBlock;
             // both CTAs' copies of this block complete on the even CTA's barrier
-            if (leader) mbar_arrive_expect_tx(&ring_full[slot], 2 * kHalfBlock);
-            const uint32_t fb = mapa_shared(smem_u32(&ring_full[slot]), 0);
-            switch (i) {
-              case 0: tma_load_3d_pair(dst, &tmKn, fb, 0, k0 + kh, bh); break;
-              case 1: tma_load_3d_pair(dst, &tmKn, fb, 64, k0 + kh, bh); break;
-              case 2: tma_load_3d_pair(dst, &tmKp, fb, 0, k0 + kh, b); break;
-              default: tma_load_3d_pair(dst, &tmV, fb, kh, k0 + (i - 3) * 64, bh); break;
+            if (leader) mbar_arrive_expect_tx(&full[slot], 2 * kHalfBlock);
+            const uint32_t fb = mapa_shared(smem_u32(&full[slot]), 0);
+            if (kprod) {
+              if (i < 2) tma_load_3d_pair(dst, &tmKn, fb, 64 * i, k0 + kh, bh);
+              else tma_load_3d_pair(dst, &tmKp, fb, 0, k0 + kh, b);
+            } else {
+              tma_load_3d_pair(dst, &tmV, fb, kh, k0 + 64 * i, bh);
             }
-            n_issued = s + 1;
+            n_issued[kprod ? 0 : 1] = s + 1;
           }
         }
       }
@@ -1068,18 +1096,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
     if (lane == 0 && leader && n_total > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(2 * kBQ, kBKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(2 * kBQ, kDV, false, true);
-      const uint32_t ring0 = smem_u32(smem + kOffRingPair);
+      const uint32_t kring0 = smem_u32(smem + kOffKRing);
+      const uint32_t vring0 = smem_u32(smem + kOffVRing);
       const uint32_t o_tmem = tmem_base + kColOPair;
       const int n0 = items.n_visit[0];  // the first item's tiles come first
       bool ok = true;
       bool issued_any = false;
       uint32_t q_ready = 0;
-      auto block_addr = [&](uint32_t seq) { return ring0 + (seq % kRingPair) * kHalfBlock; };
-      auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
-        return mbar_wait(&ring_full[seq % kRingPair], (seq / kRingPair) & 1u, ctl, site);
+      auto k_addr = [&](uint32_t seq) { return kring0 + (seq % kKRing) * kHalfBlock; };
+      auto v_addr = [&](uint32_t seq) { return vring0 + (seq % kVRing) * kHalfBlock; };
+      auto wait_k = [&](uint32_t seq) -> bool {
+        return mbar_wait(&k_full[seq % kKRing], (seq / kKRing) & 1u, ctl, 13);
       };
-      auto release = [&](uint32_t seq) {
-        mma_commit_pair_mc(&ring_empty[seq % kRingPair], kPairMask);
+      auto wait_v = [&](uint32_t seq) -> bool {
+        return mbar_wait(&v_full[seq % kVRing], (seq / kVRing) & 1u, ctl, 12);
       };
       auto issue_s = [&](int j) -> bool {
         const int it = j < n0 ? 0 : 1;
@@ -1091,9 +1121,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
           if (kRope && !mbar_wait(&q_rot[it], 0, ctl, 16)) return false;
           q_ready |= 1u << it;
         }
-        const uint32_t base = uint32_t(j) * kBlocksPerTilePair;
-        if (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13))
-          return false;
+        const uint32_t base = uint32_t(j) * kKPerTile;
+        if (!wait_k(base) || !wait_k(base + 1) || !wait_k(base + 2)) return false;
         tc_fence_after();
         const uint32_t sQ = smem_u32(smem + it * kQBytes);
         const uint32_t s_tmem = tmem_base + 128u * uint32_t(j % kSBufs);
@@ -1102,25 +1131,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
-            const uint64_t kd = sdesc_sw128(block_addr(base + blk) + kk * 32, 16, 1024);
+            const uint64_t kd = sdesc_sw128(k_addr(base + blk) + kk * 32, 16, 1024);
             mma_ss_pair(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
           }
         }
         issued_any = true;
         mma_commit_pair_mc(&s_full[j % kSBufs], kPairMask);
-        release(base);
-        release(base + 1);
-        release(base + 2);
+        for (uint32_t i = 0; i < uint32_t(kKPerTile); ++i)
+          mma_commit_pair_mc(&k_empty[(base + i) % kKRing], kPairMask);
         return true;
       };
       for (int j = 0; ok && j < min(n_total, kSBufs); ++j) ok = issue_s(j);
       for (int j = 0; ok && j < n_total; ++j) {
         const int it = j < n0 ? 0 : 1;
         const int first = it == 0 ? 0 : n0;  // the item's first tile overwrites O
-        const uint32_t base = uint32_t(j) * kBlocksPerTilePair;
+        const uint32_t vbase = uint32_t(j) * kVPerTile;
         // (acquire at cluster scope: the odd CTA's P is forwarded by a remote arrive)
         if (!mbar_wait_cluster_sleep(&p_full[j % kSBufs], uint32_t(j / kSBufs) & 1u, ctl, 11) ||
-            !wait_block(base + 3, 12) || !wait_block(base + 4, 12)) {
+            !wait_v(vbase) || !wait_v(vbase + 1)) {
           ok = false;
           break;
         }
@@ -1130,7 +1158,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         const uint32_t p_tmem = tmem_base + 128u * uint32_t(j % kSBufs);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const uint32_t vb = block_addr(base + 3 + half);
+          const uint32_t vb = v_addr(vbase + half);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (j > first || half > 0 || kk > 0) ? 1u : 0u;
@@ -1140,8 +1168,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
         }
         mma_commit_pair_mc(&pv_done[j % kSBufs], kPairMask);
         if (j == first + items.n_visit[it] - 1) mma_commit_pair_mc(&o_final, kPairMask);
-        release(base + 3);
-        release(base + 4);
+        mma_commit_pair_mc(&v_empty[vbase % kVRing], kPairMask);
+        mma_commit_pair_mc(&v_empty[(vbase + 1) % kVRing], kPairMask);
         if (j + kSBufs < n_total && !issue_s(j + kSBufs)) { ok = false; break; }
       }
       if (!ok && issued_any) {
@@ -1438,15 +1466,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
   __syncwarp();
   tc_fence_before();
   cluster_sync();
-  if (leader && warp == 0 && lane == 0 && n_total > 0) {
-    // Every ring copy completes on this CTA's barriers. Account for a block
-    // that only one CTA issued (possible only after an abort), then wait for
-    // the last phase of every slot; each slot has at most one phase pending.
-    const uint32_t n_own = n_issued;
-    const uint32_t n_peer = ld_shared_cluster_u32(mapa_shared(smem_u32(&n_issued), 1));
+  if (leader && (warp == 0 || warp == 3) && lane == 0 && n_total > 0) {
+    // Every ring copy completes on this CTA's barriers (warp 0: the K ring,
+    // warp 3: the V ring). Account for a block that only one CTA issued
+    // (possible only after an abort), then wait for the last phase of every
+    // slot; each slot has at most one phase pending.
+    const int which = warp == 0 ? 0 : 1;
+    uint64_t* full = which == 0 ? k_full : v_full;
+    const uint32_t ring = which == 0 ? kKRing : kVRing;
+    const uint32_t n_own = n_issued[which];
+    const uint32_t n_peer = ld_shared_cluster_u32(mapa_shared(smem_u32(&n_issued[which]), 1));
     const uint32_t lo = min(n_own, n_peer), hi = max(n_own, n_peer);
     for (uint32_t seq = lo; seq < hi; ++seq) {
-      uint64_t* fb = &ring_full[seq % kRingPair];
+      uint64_t* fb = &full[seq % ring];
       if (seq < n_own)  // armed for both CTAs' bytes, the odd CTA's copy never came
         mbar_complete_tx_cluster(mapa_shared(smem_u32(fb), 0), kHalfBlock);
       else              // the odd CTA's copy came, this CTA never armed the phase
@@ -1454,9 +1486,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsPair, 1)
     }
     int zero = 0;
     WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
-    const uint32_t first = hi > uint32_t(kRingPair) ? hi - kRingPair : 0;
+    const uint32_t first = hi > ring ? hi - ring : 0;
     for (uint32_t seq = first; seq < hi; ++seq)
-      mbar_wait(&ring_full[seq % kRingPair], (seq / kRingPair) & 1u, drain, 3);
+      mbar_wait(&full[seq % ring], (seq / ring) & 1u, drain, 3);
   }
   // Second barrier: no copy is in flight toward either CTA; neither leaves,
   // nor frees the pair's tensor memory, before both get here.
@@ -1548,8 +1580,8 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Which kernel runs the causal and valid-length calls: MLA_ATTN_KERNEL=pair
-// (read once) selects the CTA-pair kernel, anything else the one-SM kernel.
+// Which attention kernel runs: MLA_ATTN_KERNEL=pair (read once) selects the
+// CTA-pair kernel, anything else the one-SM kernel.
 bool pair_kernel_selected() {
   static const bool v = [] {
     const char* s = std::getenv("MLA_ATTN_KERNEL");
@@ -1599,19 +1631,25 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   if (mask && valid_len) return cudaErrorInvalidValue;
   CUtensorMap tmQn, tmQp, tmKn, tmKp, tmV;
   const int BH = B * kH;
-  if (!mask && pair_kernel_selected()) {
+  if (pair_kernel_selected()) {
     // CTA pairs: K maps with 64-key boxes (each CTA loads half the keys)
     if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
         !make_map_3d(&tmKn, k_nope, kDN, T, BH, 64) || !make_map_3d(&tmKp, k_pe, kDR, T, B, 64) ||
         !make_map_3d(&tmV, v, kDV, T, BH, 64))
       return cudaErrorInvalidValue;
-    auto kern = rope_cs ? mla_attn_prefill_pair_kernel<false, true>
-                        : mla_attn_prefill_pair_kernel<false, false>;
-    static ContextCache pair_attr[2];
+    auto kern = mask ? (rope_cs ? mla_attn_prefill_pair_kernel<true, true>
+                                : mla_attn_prefill_pair_kernel<true, false>)
+                     : (rope_cs ? mla_attn_prefill_pair_kernel<false, true>
+                                : mla_attn_prefill_pair_kernel<false, false>);
+    static ContextCache pair_attr[4];
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemPairBytes),
-                                     &pair_attr[rope_cs ? 1 : 0]);
+                                     &pair_attr[(mask ? 1 : 0) + (rope_cs ? 2 : 0)]);
     if (e != cudaSuccess) return e;
     AttnArgs a{};
+    a.mask = static_cast<const __nv_bfloat16*>(mask);
+    a.mask_ld = mask_ld;
+    a.mask_vec = mask_rows_vec_ok(mask, mask_ld) ? 1 : 0;
+    a.tile_class = static_cast<const uint8_t*>(tile_class);
     a.valid_len = valid_len;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.B = B;
