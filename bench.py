@@ -473,9 +473,11 @@ def run_ours(args, w, rank, world, local_rank):
     o_avg = statistics.mean(oproj_ms)
     g_avg = statistics.mean(gemm_ms)
     small_m = B * T <= SMALL_M_MAX and not fp8
-    # causal and valid-length calls run on CTA pairs when MLA_ATTN_KERNEL=pair
+    # MLA_ATTN_KERNEL=pair runs every attention call on CTA pairs; otherwise
+    # the one-SM kernel runs (half-tile scores for causal and valid-length
+    # calls unless MLA_ATTN_KERNEL=tile)
     attn_kernel = ("mla_attn_prefill_pair_kernel"
-                   if not dense_mask and os.environ.get("MLA_ATTN_KERNEL") == "pair"
+                   if os.environ.get("MLA_ATTN_KERNEL") == "pair"
                    else "mla_attn_prefill_kernel")
     kern = {"attn": (fa, a_avg, "attn_prefill.cu", attn_kernel),
             "oproj": (fo, g_avg, "fp8_oproj.cu" if fp8 else "oproj_gemm.cu",

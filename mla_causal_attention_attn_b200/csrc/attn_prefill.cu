@@ -40,6 +40,16 @@
 //                all-zero tiles of an explicit mask) take a single pass
 //                against the running max; the others two passes.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
+//
+// Half-tile scores (causal and valid-length calls): with 128-key tiles a
+// query tile's chain S_j -> softmax_j -> PV_j -> S_{j+1} is serial, and the
+// tensor pipe idles whenever both softmax warpgroups are busy. There each
+// 128-column S buffer is split into two 64-key buffers, and an issuer runs
+// S(0), S(1), then PV(u), S(u+2) for every 64-key half tile u, so the scores
+// of the next half tile are computed while the softmax works on this one;
+// the softmax waits for PV(u-1) only before it rescales O. The O accumulators
+// and the K/V ring are unchanged. Explicit masks keep 128-key tiles (a query
+// tile there may skip key tiles in the middle of the visited ones).
 #include "attn_prefill.h"
 
 #include <cstdlib>
@@ -200,13 +210,13 @@ struct ScoreChunk {
   }
 };
 
-// Maximum of a row of 128 raw scores; on the diagonal tile keys c > r are
-// excluded (causal).
-template <bool kDiag>
-__device__ __forceinline__ float raw_row_max(const uint32_t (&raw)[kBKV], int r) {
+// Maximum of a row of W (128 or 64) raw scores; on the diagonal tile keys
+// c > r are excluded (causal).
+template <bool kDiag, int W = kBKV>
+__device__ __forceinline__ float raw_row_max(const uint32_t (&raw)[W], int r) {
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int i = 0; i < kBKV; i += 8) {
+  for (int i = 0; i < W; i += 8) {
     float v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -249,18 +259,178 @@ __device__ __forceinline__ void p_chunk_causal(const uint32_t* raw, int c, int r
   }
 }
 
-template <bool kMasked, bool kRope>
+// One softmax step of a query row (one thread, one TMEM lane) over kW keys:
+// a 128-key tile, or a 64-key half tile. Reads the raw scores at TMEM column
+// colS, folds them into the running max m (log2 units) and the running sum
+// l, writes P as bf16 over the first kW / 2 columns, and rescales O (column
+// colO) when the max grew past the headroom. Tiles that need no mask entries
+// added (fast_route: every causal tile, the all-zero, causal-pattern and
+// prefix tiles of an explicit mask; positive scale) take a single pass
+// against the running max; keys c > lim are excluded there when diag is set.
+// The others, and the first tile, take two passes through sc. False when a
+// bounded wait gave up.
+template <bool kMasked, int kW>
+__device__ __forceinline__ bool softmax_step(const AttnArgs& args, uint32_t lane_base,
+                                             uint32_t colS, uint32_t colO,
+                                             const ScoreChunk<kMasked>& sc, bool fast_route,
+                                             bool diag, int lim, int r, uint32_t n, float& m,
+                                             float& l, uint64_t* pv_bar, uint32_t pv_par,
+                                             const WaitCtl& ctl) {
+  constexpr int kC = kW / 32;  // 32-key chunks
+  static_assert(kW == 64 || kW == kBKV, "tile width");
+  uint32_t raw[kW];
+#pragma unroll
+  for (int c = 0; c < kC; ++c)
+    tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
+  tmem_ld_wait();
+  reg_fence(raw);
+  float alpha = 1.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
+  // Fast-route tiles after the first: one pass against the running max m,
+  // writing P (64 keys per store). Every p is then <= 2^8 unless the max
+  // grew by more than the headroom, so a row sum <= 2^8 proves no rescale
+  // is due; otherwise (rare: many keys near the max, or a new max) the
+  // tile's true max is taken and, only if it grew past the headroom, the
+  // tile is redone exactly below (new max, O rescaled). The first tile and
+  // the tiles that need their mask entries added take the exact two-pass
+  // route. The choice is warp-uniform (a row whose max is still -inf fails
+  // the row-sum test).
+  bool exact = !(fast_route && n > 0);
+  float rowsum = 0.f;
+  if (!exact) {
+#pragma unroll
+    for (int c2 = 0; c2 < kC; c2 += 2) {
+      uint32_t pk[32];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
+        if (diag)
+          p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, lim, args.scale_log2, m, ph,
+                               acc);
+        else
+          p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph,
+                                acc);
+      }
+      tmem_st32(lane_base + colS + 16 * c2, pk);
+    }
+    rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    if (__any_sync(0xffffffffu, !(rowsum <= 256.f))) {
+      const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
+                       args.scale_log2;
+      exact = __any_sync(0xffffffffu, !(mt <= m + kRescaleThreshold));
+      if (exact) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      }
+    }
+  }
+  if (exact) {
+    float mt;
+    if (fast_route) {
+      // positive scale: the maximum of the raw scores gives the maximum of
+      // the scaled ones
+      mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
+      mt *= args.scale_log2;
+    } else {
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        float x[32];
+        sc.apply(raw + c * 32, c, args.scale_log2, 0.f, x);
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          m4[0] = fmax3(m4[0], x[i], x[i + 1]);
+          m4[1] = fmax3(m4[1], x[i + 2], x[i + 3]);
+          m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
+          m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
+        }
+        // keep the scaled, masked scores: the exponentials below need
+        // neither the mask nor the scale again
+#pragma unroll
+        for (int i = 0; i < 32; ++i) raw[c * 32 + i] = __float_as_uint(x[i]);
+      }
+      mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    }
+    float m_new = m;
+    if (n == 0) {
+      m_new = mt;
+    } else if (mt > m + kRescaleThreshold) {
+      m_new = mt;
+      alpha = fast_exp2(m - m_new);
+    }
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+    m = m_new;
+
+    // P as bf16 pairs over the first kW / 2 columns of the S buffer (every
+    // score is in registers by now), 32 keys per store.
+#pragma unroll
+    for (int c = 0; c < kC; ++c) {
+      const uint32_t* rc = raw + c * 32;
+      uint32_t pk[16];
+      if (fast_route) {
+        if (diag)
+          p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
+        else
+          p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
+      } else {
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(rc[i]) - m_use;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(x[2 * i]);
+          const float p1 = fast_exp2(x[2 * i + 1]);
+          fadd2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)],
+                acc[2 * (i & 3) + 1], p0, p1);
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+      }
+      tmem_st16(lane_base + colS + 16 * c, pk);
+    }
+    rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+
+    // The rescale needs O to hold P_{n-1} V_{n-1}. On 128-key tiles that PV
+    // was issued before this S, and the commit behind s_full covers every
+    // earlier MMA (pv_bar null); on half tiles it is issued after this S and
+    // its own commit (pv_bar) is awaited. The rescale lands before PV_n, which
+    // waits for p_full. (Only the exact route can change the max.)
+    if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (pv_bar) {
+        if (!mbar_wait_warp(pv_bar, pv_par, ctl, 23)) return false;
+        tc_fence_after();
+      }
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(lane_base + colO + c * 32, rr);
+        tmem_ld_wait();
+        reg_fence(rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+        tmem_st32(lane_base + colO + c * 32, rr);
+      }
+    }
+  }  // exact
+  l = l * alpha + rowsum;
+  return true;
+}
+
+template <bool kMasked, bool kRope, bool kHalf>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQn,
                             const __grid_constant__ CUtensorMap tmQp,
                             const __grid_constant__ CUtensorMap tmKn,
                             const __grid_constant__ CUtensorMap tmKp,
                             const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+  static_assert(!(kMasked && kHalf), "half-tile scores serve the causal kernel only");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[2];     // query tile i is in shared memory
   __shared__ uint64_t q_rot[2];      // its rotary part is rotated (rotary calls only)
   __shared__ uint64_t ring_full[kRing], ring_empty[kRing];
-  __shared__ uint64_t s_full[2], p_full[2];
+  // S ready / P written: [query tile] on 128-key tiles, [2 * query tile +
+  // half] on half tiles
+  __shared__ uint64_t s_full[4], p_full[4];
+  __shared__ uint64_t pv_done[2];   // half tiles: a PV product of query tile i completed
   __shared__ uint64_t o_final[2];
   __shared__ uint64_t drain_bar[2];
   __shared__ uint64_t s_issued[2];  // issuer i has issued (or skipped) S of its next tile
@@ -313,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // released once by each query tile's MMA issuer
       mbar_init(&ring_empty[s], tiles.exists[1] ? 2 : 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
     }
@@ -321,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_final[i], 1);
       mbar_init(&drain_bar[i], 1);
       mbar_init(&s_issued[i], 1);
+      mbar_init(&pv_done[i], 1);
       mbar_init(&never_bar, 1);
     }
     fence_barrier_init();
@@ -444,11 +615,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&q_full[qi], 0, ctl, 10);
       if (kRope && ok) ok = mbar_wait(&q_rot[qi], 0, ctl, 16);
       bool issued_any = false;
-      uint32_t n_pv = 0;       // PVs issued
-      uint32_t n_tiles = 0;    // visited key tiles so far
-      int prev = -1;           // previous visited key tile
-      bool prev_act = false;   // did this query tile use it
-      uint32_t prev_base = 0;  // block sequence number of prev's first block
 
       auto wait_block = [&](uint32_t seq, uint32_t site) -> bool {
         return mbar_wait(&ring_full[seq % kRing], (seq / kRing) & 1u, ctl, site);
@@ -464,77 +630,155 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&ring_empty[seq % kRing]);
       };
-      // O += P V for the previous key tile, then release its two V blocks.
-      auto finish_prev = [&]() -> bool {
-        if (!wait_block(prev_base + 3, 12) || !wait_block(prev_base + 4, 12)) return false;
-        if (prev_act) {
-          if (!mbar_wait(&p_full[qi], n_pv & 1u, ctl, 11)) return false;
+      if constexpr (kHalf) {
+        // Half tiles: sub-tile u = 2 kt + hb is keys kt*128 + 64 hb .. +63 of
+        // this query tile's active key tiles 0 .. n_act-1 (a prefix of the
+        // visited ones); its scores go to buffer hb (64 TMEM columns, P over
+        // the first 32). Order: S(0), S(1), then for each u: PV(u), S(u+2),
+        // so the scores of the next half tile are ready while the softmax
+        // works on this one. S(u+2) reuses the buffer PV(u) reads; the tensor
+        // pipe runs one thread's MMAs in order.
+        constexpr uint32_t idesc_sh = idesc_bf16_f32(kBQ, kBKV / 2, false, false);
+        const int n_act = min(tiles.qt[qi] + 1, tiles.end);
+        const int n_sub = 2 * n_act;
+        auto issue_s = [&](int u) -> bool {
+          const int kt = u >> 1, hb = u & 1;
+          const uint32_t base = kBlocksPerTile * uint32_t(kt);
+          if (hb == 0 &&
+              (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13)))
+            return false;
           tc_fence_after();
-          // Each V block holds 64 keys x 128 value dims, MN-major: value dims
-          // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB
-          // apart (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t vb = block_addr(prev_base + 3 + half);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (n_pv > 0 || half > 0 || kk > 0) ? 1u : 0u;
-              const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
-              mma_ts(o_tmem, s_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
-            }
-          }
-          ++n_pv;
-          issued_any = true;
-        }
-        release(prev_base + 3, prev_act);
-        release(prev_base + 4, prev_act);
-        return true;
-      };
-
-      uint32_t base = 0;
-      for (int kt = tiles.first(); ok && kt < tiles.end;
-           kt = tiles.next(kt), base += kBlocksPerTile, ++n_tiles) {
-        const bool act = tiles.active(qi, kt);
-        if (prev >= 0 && !finish_prev()) { ok = false; break; }
-        if (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13)) {
-          ok = false;
-          break;
-        }
-        // S order: tile 1 waits for tile 0's S of this key tile, tile 0 for
-        // tile 1's S of the previous one.
-        if (pair) {
-          if (qi == 1) {
-            if (!mbar_wait(&s_issued[0], n_tiles & 1u, ctl, 15)) { ok = false; break; }
-          } else if (n_tiles > 0) {
-            if (!mbar_wait(&s_issued[1], (n_tiles - 1) & 1u, ctl, 15)) { ok = false; break; }
-          }
-        }
-        if (act) {
-          tc_fence_after();
-          const uint32_t k_addr[3] = {block_addr(base), block_addr(base + 1),
-                                      block_addr(base + 2)};
+          const uint32_t s_buf = s_tmem + 64 * hb;
 #pragma unroll
           for (int blk = 0; blk < 3; ++blk) {
+            const uint32_t kb = block_addr(base + blk) + hb * (kBlock / 2);  // keys 64 hb ..
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
-              const uint64_t kd = sdesc_sw128(k_addr[blk] + kk * 32, 16, 1024);
-              mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
+              const uint64_t kd = sdesc_sw128(kb + kk * 32, 16, 1024);
+              mma_ss(s_buf, qd, kd, idesc_sh, (blk | kk) != 0 ? 1u : 0u);
             }
           }
           issued_any = true;
-          mma_commit(&s_full[qi]);
+          mma_commit(&s_full[2 * qi + hb]);
+          if (hb == 1) {  // both halves read the K blocks
+            release(base, true);
+            release(base + 1, true);
+            release(base + 2, true);
+          }
+          return true;
+        };
+        // O += P V over the 64 keys of one V block, then release it.
+        auto issue_pv = [&](int u) -> bool {
+          const int kt = u >> 1, hb = u & 1;
+          const uint32_t vseq = kBlocksPerTile * uint32_t(kt) + 3 + hb;
+          if (!wait_block(vseq, 12)) return false;
+          if (!mbar_wait(&p_full[2 * qi + hb], uint32_t(u >> 1) & 1u, ctl, 11)) return false;
+          tc_fence_after();
+          const uint32_t vb = block_addr(vseq);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
+            mma_ts(o_tmem, s_tmem + 64 * hb + kk * 8, vd, idesc_o, (u | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&pv_done[qi]);
+          release(vseq, true);
+          return true;
+        };
+        if (ok) ok = issue_s(0);
+        if (ok) ok = issue_s(1);
+        for (int u = 0; ok && u < n_sub; ++u) {
+          ok = issue_pv(u);
+          if (ok && u + 2 < n_sub) ok = issue_s(u + 2);
         }
-        if (pair) mbar_arrive(&s_issued[qi]);
-        release(base, act);
-        release(base + 1, act);
-        release(base + 2, act);
-        prev = kt;
-        prev_act = act;
-        prev_base = base;
+        if (ok) mma_commit(&o_final[qi]);
+        // The visited key tile past this query tile's last one (causal: the
+        // other query tile's diagonal) is released unused, block by block
+        // once it has landed, after every block this tile used.
+        for (int kt = n_act; ok && kt < tiles.end; ++kt)
+          for (uint32_t i = 0; ok && i < uint32_t(kBlocksPerTile); ++i) {
+            const uint32_t seq = kBlocksPerTile * uint32_t(kt) + i;
+            ok = wait_block(seq, 13);
+            if (ok) release(seq, false);
+          }
+      } else {
+        uint32_t n_pv = 0;       // PVs issued
+        uint32_t n_tiles = 0;    // visited key tiles so far
+        int prev = -1;           // previous visited key tile
+        bool prev_act = false;   // did this query tile use it
+        uint32_t prev_base = 0;  // block sequence number of prev's first block
+        // O += P V for the previous key tile, then release its two V blocks.
+        auto finish_prev = [&]() -> bool {
+          if (!wait_block(prev_base + 3, 12) || !wait_block(prev_base + 4, 12)) return false;
+          if (prev_act) {
+            if (!mbar_wait(&p_full[qi], n_pv & 1u, ctl, 11)) return false;
+            tc_fence_after();
+            // Each V block holds 64 keys x 128 value dims, MN-major: value dims
+            // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB
+            // apart (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t vb = block_addr(prev_base + 3 + half);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t acc = (n_pv > 0 || half > 0 || kk > 0) ? 1u : 0u;
+                const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
+                mma_ts(o_tmem, s_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
+              }
+            }
+            ++n_pv;
+            issued_any = true;
+          }
+          release(prev_base + 3, prev_act);
+          release(prev_base + 4, prev_act);
+          return true;
+        };
+
+        uint32_t base = 0;
+        for (int kt = tiles.first(); ok && kt < tiles.end;
+             kt = tiles.next(kt), base += kBlocksPerTile, ++n_tiles) {
+          const bool act = tiles.active(qi, kt);
+          if (prev >= 0 && !finish_prev()) { ok = false; break; }
+          if (!wait_block(base, 13) || !wait_block(base + 1, 13) || !wait_block(base + 2, 13)) {
+            ok = false;
+            break;
+          }
+          // S order: tile 1 waits for tile 0's S of this key tile, tile 0 for
+          // tile 1's S of the previous one.
+          if (pair) {
+            if (qi == 1) {
+              if (!mbar_wait(&s_issued[0], n_tiles & 1u, ctl, 15)) { ok = false; break; }
+            } else if (n_tiles > 0) {
+              if (!mbar_wait(&s_issued[1], (n_tiles - 1) & 1u, ctl, 15)) { ok = false; break; }
+            }
+          }
+          if (act) {
+            tc_fence_after();
+            const uint32_t k_addr[3] = {block_addr(base), block_addr(base + 1),
+                                        block_addr(base + 2)};
+#pragma unroll
+            for (int blk = 0; blk < 3; ++blk) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t qd = sdesc_sw128(sQ + blk * kBlock + kk * 32, 16, 1024);
+                const uint64_t kd = sdesc_sw128(k_addr[blk] + kk * 32, 16, 1024);
+                mma_ss(s_tmem, qd, kd, idesc_s, (blk | kk) != 0 ? 1u : 0u);
+              }
+            }
+            issued_any = true;
+            mma_commit(&s_full[qi]);
+          }
+          if (pair) mbar_arrive(&s_issued[qi]);
+          release(base, act);
+          release(base + 1, act);
+          release(base + 2, act);
+          prev = kt;
+          prev_act = act;
+          prev_base = base;
+        }
+        if (ok && prev >= 0) ok = finish_prev();
+        if (ok && n_pv > 0) mma_commit(&o_final[qi]);
       }
-      if (ok && prev >= 0) ok = finish_prev();
-      if (ok && n_pv > 0) mma_commit(&o_final[qi]);
       if (!ok && issued_any) {
         mma_commit(&drain_bar[qi]);
         int zero = 0;
@@ -598,182 +842,104 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY;  // running max, log2 units
     float l = 0.f;        // running sum of p (fp32, unrounded)
     uint32_t n = 0;
-    for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) {
-      if (!tiles.active(wi, kt)) continue;
-      const int k0 = kt * kBKV;
-      // Failure-detection test: query tile 0 of the first CTA waits on a
-      // barrier nothing arrives on; the bounded wait must time out, abort the
-      // CTA cleanly and report through the status word.
-      if (args.test_stall && wi == 0 && blockIdx.x == 0 &&
-          !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
-        ok = false;
-        break;
-      }
-      if (!mbar_wait_warp(&s_full[wi], n & 1u, ctl, 20)) { ok = false; break; }
-      tc_fence_after();
-      // The 128 scores of this thread's row are read from tensor memory once
-      // and kept in registers for both passes (row maximum, exponentials).
-      ScoreChunk<kMasked> sc;
-      sc.cls = (kMasked && row_valid)
-                   ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed))
-                   : uint8_t(kTileZero);
-      sc.row_valid = row_valid;
-      sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
-      sc.kvalid = args.T - k0;
-      sc.mask_vec = args.mask_vec;
-      // The fast route (scores need no mask add): every tile of the causal
-      // kernel, and the all-zero and causal-pattern tiles of an explicit
-      // mask. It needs a positive scale (the raw maximum is then the scaled
-      // one).
-      const uint8_t tile_cls =
-          kMasked ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed)) : uint8_t(kTileZero);
-      const bool causal_tile = !kMasked ? kt == qt : tile_cls == kTileCausal;
-      const bool prefix_tile = kMasked && tile_cls >= kTilePrefix;
-      const bool fast_route =
-          (tile_cls == kTileZero || tile_cls == kTileCausal || prefix_tile) &&
-          args.scale_log2 > 0.f;
-      // Keys c <= lim of the tile are allowed on the fast route: c <= r on a
-      // causal diagonal tile, c <= the class's limit on a prefix tile, and
-      // none at or past the sequence's key count (T, or valid_len[b]). `diag`
-      // marks the tiles where that limit cuts (warp-uniform).
-      const int key_end = kMasked ? args.T : n_keys;
-      const bool diag = causal_tile || prefix_tile || key_end - k0 < kBKV;
-      const int lim = min(causal_tile ? r : (prefix_tile ? int(tile_cls) - kTilePrefix : kBKV - 1),
-                          key_end - 1 - k0);
-      sc.diag_row = (kMasked ? (causal_tile || prefix_tile) : diag) ? lim : kBKV;
-      uint32_t raw[kBKV];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_base + colS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
-      tmem_ld_wait();
-      reg_fence(raw);
-      float alpha = 1.f;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 paired partial sums
-      // Fast-route tiles after the first: one pass against the running max m,
-      // writing P (64 keys per store). Every p is then <= 2^8 unless the max
-      // grew by more than the headroom, so a row sum <= 2^8 proves no rescale
-      // is due; otherwise (rare: many keys near the max, or a new max) the
-      // tile's true max is taken and, only if it grew past the headroom, the
-      // tile is redone exactly below (new max, O rescaled). The first tile and
-      // the tiles that need their mask entries added take the exact two-pass
-      // route. The choice is warp-uniform (a row whose max is still -inf fails
-      // the row-sum test).
-      bool exact = !(fast_route && n > 0);
-      float rowsum = 0.f;
-      if (!exact) {
-#pragma unroll
-        for (int c2 = 0; c2 < 4; c2 += 2) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t(&ph)[16] = *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * h2);
-            if (diag)
-              p_chunk_causal<true>(raw + (c2 + h2) * 32, c2 + h2, lim, args.scale_log2, m, ph,
-                                   acc);
-            else
-              p_chunk_causal<false>(raw + (c2 + h2) * 32, c2 + h2, r, args.scale_log2, m, ph,
-                                    acc);
-          }
-          tmem_st32(lane_base + colS + 16 * c2, pk);
+    if constexpr (kHalf) {
+      // Half tiles (causal kernel): 64 keys per step, the two score buffers
+      // of this query tile in turn.
+      const int n_sub = (has_work && tiles.exists[wi]) ? 2 * min(qt + 1, tiles.end) : 0;
+      for (int u = 0; u < n_sub; ++u) {
+        const int kt = u >> 1, hb = u & 1;
+        const int k0 = kt * kBKV + 64 * hb;
+        if (args.test_stall && wi == 0 && blockIdx.x == 0 &&
+            !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
+          ok = false;
+          break;
         }
-        rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        if (__any_sync(0xffffffffu, !(rowsum <= 256.f))) {
-          const float mt = (diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r)) *
-                           args.scale_log2;
-          exact = __any_sync(0xffffffffu, !(mt <= m + kRescaleThreshold));
-          if (exact) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-          }
+        if (!mbar_wait_warp(&s_full[2 * wi + hb], uint32_t(u >> 1) & 1u, ctl, 20)) {
+          ok = false;
+          break;
         }
-      }
-      if (exact) {
-      float mt;
-      if (fast_route) {
-        // positive scale: the maximum of the raw scores gives the maximum of
-        // the scaled ones
-        mt = diag ? raw_row_max<true>(raw, lim) : raw_row_max<false>(raw, r);
-        mt *= args.scale_log2;
-      } else {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float x[32];
-          sc.apply(raw + c * 32, c, args.scale_log2, 0.f, x);
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            m4[0] = fmax3(m4[0], x[i], x[i + 1]);
-            m4[1] = fmax3(m4[1], x[i + 2], x[i + 3]);
-            m4[2] = fmax3(m4[2], x[i + 4], x[i + 5]);
-            m4[3] = fmax3(m4[3], x[i + 6], x[i + 7]);
-          }
-          // keep the scaled, masked scores: the exponentials below need
-          // neither the mask nor the scale again
-#pragma unroll
-          for (int i = 0; i < 32; ++i) raw[c * 32 + i] = __float_as_uint(x[i]);
+        tc_fence_after();
+        // keys c <= lim of the half tile: c + 64 hb <= r on the diagonal tile
+        // (none for rows r < 64 in its second half), and none at or past the
+        // sequence's key count
+        const bool causal_tile = kt == qt;
+        const bool diag = causal_tile || n_keys - k0 < kBKV / 2;
+        const int lim = min(causal_tile ? r - 64 * hb : kBKV / 2 - 1, n_keys - 1 - k0);
+        ScoreChunk<kMasked> sc;
+        sc.cls = kTileZero;
+        sc.row_valid = row_valid;
+        sc.mrow = nullptr;
+        sc.kvalid = args.T - k0;
+        sc.mask_vec = 0;
+        sc.diag_row = diag ? lim : kBKV;
+        // Before rescaling O the step waits for PV(u-1): at most one PV of
+        // this query tile is outstanding here (S(u), awaited above, was issued
+        // after PV(u-2)), so the parity of pv_done is unambiguous.
+        if (!softmax_step<kMasked, kBKV / 2>(args, lane_base, colS + 64 * hb, colO, sc,
+                                             args.scale_log2 > 0.f, diag, lim, r, n, m, l,
+                                             &pv_done[wi], (n - 1) & 1u, ctl)) {
+          ok = false;
+          break;
         }
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * wi + hb]);
+        ++n;
       }
-      float m_new = m;
-      if (n == 0) {
-        m_new = mt;
-      } else if (mt > m + kRescaleThreshold) {
-        m_new = mt;
-        alpha = fast_exp2(m - m_new);
-      }
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      m = m_new;
-
-      // P as bf16 pairs over the first 64 columns of the S buffer (every score
-      // is in registers by now), 32 keys per store.
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t* rc = raw + c * 32;
-        uint32_t pk[16];
-        if (fast_route) {
-          if (diag)
-            p_chunk_causal<true>(rc, c, lim, args.scale_log2, m_use, pk, acc);
-          else
-            p_chunk_causal<false>(rc, c, r, args.scale_log2, m_use, pk, acc);
-        } else {
-          float x[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(rc[i]) - m_use;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(x[2 * i]);
-            const float p1 = fast_exp2(x[2 * i + 1]);
-            fadd2(acc[2 * (i & 3)], acc[2 * (i & 3) + 1], acc[2 * (i & 3)],
-                  acc[2 * (i & 3) + 1], p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
-          }
+    } else {
+      for (int kt = tiles.first(); kt < tiles.end; kt = tiles.next(kt)) {
+        if (!tiles.active(wi, kt)) continue;
+        const int k0 = kt * kBKV;
+        // Failure-detection test: query tile 0 of the first CTA waits on a
+        // barrier nothing arrives on; the bounded wait must time out, abort the
+        // CTA cleanly and report through the status word.
+        if (args.test_stall && wi == 0 && blockIdx.x == 0 &&
+            !mbar_wait_warp(&never_bar, 0, ctl, 30)) {
+          ok = false;
+          break;
         }
-        tmem_st16(lane_base + colS + 16 * c, pk);
-      }
-      rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-
-      // O holds P_{n-1} V_{n-1} here: that PV was issued before this S, and
-      // the commit behind s_full covers every earlier MMA. The rescale lands
-      // before PV_n, which waits for p_full below. (Only the exact route can
-      // change the max.)
-      if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(lane_base + colO + c * 32, rr);
-          tmem_ld_wait();
-          reg_fence(rr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(lane_base + colO + c * 32, rr);
+        if (!mbar_wait_warp(&s_full[wi], n & 1u, ctl, 20)) { ok = false; break; }
+        tc_fence_after();
+        // The 128 scores of this thread's row are read from tensor memory once
+        // and kept in registers for both passes (row maximum, exponentials).
+        ScoreChunk<kMasked> sc;
+        sc.cls = (kMasked && row_valid)
+                     ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed))
+                     : uint8_t(kTileZero);
+        sc.row_valid = row_valid;
+        sc.mrow = mrow + (kMasked && row_valid ? k0 : 0);
+        sc.kvalid = args.T - k0;
+        sc.mask_vec = args.mask_vec;
+        // The fast route (scores need no mask add): every tile of the causal
+        // kernel, and the all-zero and causal-pattern tiles of an explicit
+        // mask. It needs a positive scale (the raw maximum is then the scaled
+        // one).
+        const uint8_t tile_cls =
+            kMasked ? (tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed)) : uint8_t(kTileZero);
+        const bool causal_tile = !kMasked ? kt == qt : tile_cls == kTileCausal;
+        const bool prefix_tile = kMasked && tile_cls >= kTilePrefix;
+        const bool fast_route =
+            (tile_cls == kTileZero || tile_cls == kTileCausal || prefix_tile) &&
+            args.scale_log2 > 0.f;
+        // Keys c <= lim of the tile are allowed on the fast route: c <= r on a
+        // causal diagonal tile, c <= the class's limit on a prefix tile, and
+        // none at or past the sequence's key count (T, or valid_len[b]). `diag`
+        // marks the tiles where that limit cuts (warp-uniform).
+        const int key_end = kMasked ? args.T : n_keys;
+        const bool diag = causal_tile || prefix_tile || key_end - k0 < kBKV;
+        const int lim = min(causal_tile ? r : (prefix_tile ? int(tile_cls) - kTilePrefix : kBKV - 1),
+                            key_end - 1 - k0);
+        sc.diag_row = (kMasked ? (causal_tile || prefix_tile) : diag) ? lim : kBKV;
+        if (!softmax_step<kMasked, kBKV>(args, lane_base, colS, colO, sc, fast_route, diag, lim, r,
+                                         n, m, l, nullptr, 0, ctl)) {
+          ok = false;
+          break;
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[wi]);
+        ++n;
       }
-      }  // exact
-      l = l * alpha + rowsum;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[wi]);
-      ++n;
     }
 
     // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]
@@ -1580,13 +1746,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Which attention kernel runs: MLA_ATTN_KERNEL=pair (read once) selects the
-// CTA-pair kernel, anything else the one-SM kernel.
+// Which attention kernel runs (MLA_ATTN_KERNEL, read once): "pair" selects
+// the CTA-pair kernel; "tile" the one-SM kernel with 128-key score tiles for
+// causal and valid-length calls too; anything else the one-SM kernel, with
+// half-tile scores for causal and valid-length calls.
+bool kernel_env_is(const char* name) {
+  const char* s = std::getenv("MLA_ATTN_KERNEL");
+  return s && std::strcmp(s, name) == 0;
+}
 bool pair_kernel_selected() {
-  static const bool v = [] {
-    const char* s = std::getenv("MLA_ATTN_KERNEL");
-    return s && std::strcmp(s, "pair") == 0;
-  }();
+  static const bool v = kernel_env_is("pair");
+  return v;
+}
+bool tile_kernel_selected() {
+  static const bool v = kernel_env_is("tile");
   return v;
 }
 
@@ -1672,13 +1845,17 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
       !make_map_3d(&tmKn, k_nope, kDN, T, BH) || !make_map_3d(&tmKp, k_pe, kDR, T, B) ||
       !make_map_3d(&tmV, v, kDV, T, BH, 64))
     return cudaErrorInvalidValue;
-  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true>
-                             : mla_attn_prefill_kernel<true, false>)
-                  : (rope_cs ? mla_attn_prefill_kernel<false, true>
-                             : mla_attn_prefill_kernel<false, false>);
-  static ContextCache attr_done[4];
+  // causal and valid-length calls: half-tile scores unless MLA_ATTN_KERNEL=tile
+  const bool half = !mask && !tile_kernel_selected();
+  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, false>
+                             : mla_attn_prefill_kernel<true, false, false>)
+                  : half ? (rope_cs ? mla_attn_prefill_kernel<false, true, true>
+                                    : mla_attn_prefill_kernel<false, false, true>)
+                         : (rope_cs ? mla_attn_prefill_kernel<false, true, false>
+                                    : mla_attn_prefill_kernel<false, false, false>);
+  static ContextCache attr_done[6];
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemBytes),
-                                   &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0)]);
+                                   &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0) + (half ? 4 : 0)]);
   if (e != cudaSuccess) return e;
   AttnArgs a;
   a.mask = static_cast<const __nv_bfloat16*>(mask);

@@ -124,6 +124,28 @@ def make_inputs(B: int, T: int, *, q_scale: float = 1.0, key_padding: bool = Fal
     return out
 
 
+def make_peaked_inputs(B: int, T: int, *, gain: float = 6.0, seed: int = 0):
+    """Inputs whose query row i points at key rows i and i+1.
+
+    Keys and values are drawn as by make_inputs. Per head, query row i is
+    gain * (key row i + key row i+1) over all 192 dims, its rotary part built
+    from the shared rotary key; the last row is 2 * gain * key row T-1. With
+    the default softmax scale the scores of keys i and i+1 then stand tens of
+    nats above the row's others, and which of the two is higher differs from
+    row to row. A check on these inputs is sharp where random ones are not:
+    under the causal mask row i's output is v_i to bf16 precision, while a
+    kernel that let key i+1 in, or kept key i out, is off by the size of v."""
+    d = make_inputs(B, T, seed=seed, with_weight=False)
+
+    def nxt(x):
+        return torch.cat([x[:, :, 1:], x[:, :, -1:]], dim=2).float()
+
+    d["q_nope"] = (gain * (d["k_nope"].float() + nxt(d["k_nope"]))).to(torch.bfloat16)
+    q_pe = gain * (d["k_pe"].float() + nxt(d["k_pe"]))
+    d["q_pe"] = q_pe.expand(B, H, T, DR).contiguous().to(torch.bfloat16)
+    return d
+
+
 def make_positions(B: int, T: int, kind: str = "arange", seed: int = 0) -> torch.Tensor:
     """position_ids [B, T] int32 for the rotary path:
     "arange"  0..T-1 in every sequence (what a None position_ids means);

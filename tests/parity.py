@@ -77,6 +77,18 @@ def assert_parity(got, ref, label: str = "") -> dict:
     return m
 
 
+def assert_peaked(got, ref, rows, label: str = "") -> None:
+    """Rows whose answer is essentially one value row (the causal rows of
+    inputs.make_peaked_inputs): every element within half a bf16 ulp of the
+    oracle, plus 1e-4 for the vanishing weight of the other keys."""
+    g = np.asarray(got, dtype=np.float64)[rows]
+    r = np.asarray(ref, dtype=np.float64)[rows]
+    err = np.abs(g - r)
+    bad = np.argwhere(err > bf16_half_ulp(r) + 1e-4)
+    assert bad.size == 0, (f"{label}: {len(bad)} elements off, first at (row, col) "
+                           f"{bad[0].tolist()}: got {g[tuple(bad[0])]} want {r[tuple(bad[0])]}")
+
+
 def sample_rows(B: int, T: int, n_random: int, seed: int = 0, valid_len=None, tile: int = 128):
     """Rows (b, t) to check at full size: t = 0 and T-1, every tile boundary
     +-1, every row of the last query tile, rows around each valid length, and

@@ -1,13 +1,27 @@
-"""The two attention kernels on the same causal inputs.
+"""The attention kernels side by side, and sharp checks of their key masks.
 
-Causal and valid-length calls run the one-SM kernel, or, in a process started
-with MLA_ATTN_KERNEL=pair, the CTA-pair kernel (one M = 256 MMA over two SMs,
-double-buffered scores). Each is run in a child process with the variable set
-accordingly. Both must match the fp64 oracle, and they must agree with each
-other: the per-row
-arithmetic (fp32 scores, the same softmax routes, P rounded to bf16, fp32
-accumulation of P V) is the same, so any difference beyond a rounding flip of
-a bf16 output would point at a layout or masking mistake in one of them.
+Causal and valid-length calls run, by MLA_ATTN_KERNEL (read once per
+process), the one-SM kernel with 64-key (half-tile) score buffers (the
+default), the same kernel on 128-key tiles ("tile", the tiles explicit masks
+always use), or the CTA-pair kernel ("pair"). Each runs here in a child
+process with the variable set. Checked:
+- every kernel against the fp64 oracle, on random inputs (causal and
+  valid_len) and on inputs whose query row i points at keys i and i+1
+  (inputs.make_peaked_inputs). On those the causal answer of row i is v_i to
+  bf16 precision, so they are compared element by element within half a bf16
+  ulp: a kernel that let key i+1 in, or kept key i out, would be off by the
+  size of v itself, at any row, tile boundary or ragged tail. The running
+  max jumps on the diagonal there, so the rescale of O is exercised too;
+- the tile and pair kernels do the same per-row arithmetic (128-key tiles,
+  the same softmax routes): equal to within one bf16 ulp;
+- the half-tile kernel against the tile kernel: rows whose allowed keys all
+  lie in the first 64 are bit-identical (the same maximum, sums and products);
+  on the other rows the running max starts from 64 keys instead of 128, so P
+  rounds differently, and their errors against the oracle are of one size;
+- on 128-key tiles an explicit causal mask gives the causal call's result bit
+  for bit, and a dense causal key-padding mask the valid_len call's outside
+  the query tile holding the last valid key (whose diagonal mask tile is
+  mixed).
 """
 import json
 import os
@@ -19,13 +33,19 @@ import pytest
 import torch
 
 import oracle
-from mla_causal_attention_attn_b200 import binding, inputs
-from parity import assert_parity, to_f64
+from mla_causal_attention_attn_b200 import inputs
+from parity import assert_parity, assert_peaked, to_f64
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 pytestmark = pytest.mark.gpu
 
 CASES = [(1, 1), (1, 130), (2, 300), (1, 1024), (3, 257)]
+PEAKED = [(1, 1), (2, 300), (1, 1024)]
+
+
+def lens_of(B, T):
+    return [max(1, T - 77 * (b + 1)) for b in range(B)]
+
 
 CHILD = r"""
 import sys, torch
@@ -33,46 +53,126 @@ sys.path.insert(0, ROOT)
 from mla_causal_attention_attn_b200 import binding, inputs
 dev = torch.device("cuda:0")
 outs = {}
-for B, T in CASES:
-    d = inputs.make_inputs(B, T, seed=1300 + T + B, with_weight=False)
+
+def run(d, tag, lens, mask=None):
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
-    outs[f"{B}x{T}"] = binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"],
-                                            g["v"], softmax_scale=g["softmax_scale"]).cpu()
-    vl = torch.tensor([max(1, T - 77 * (b + 1)) for b in range(B)], dtype=torch.int32)
-    outs[f"{B}x{T}v"] = binding.attn_prefill_varlen(g["q_nope"], g["q_pe"], g["k_nope"],
-                                                    g["k_pe"], g["v"], vl.to(dev),
-                                                    softmax_scale=g["softmax_scale"]).cpu()
+    outs[tag] = binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                     softmax_scale=g["softmax_scale"]).cpu()
+    vl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    outs[tag + "v"] = binding.attn_prefill_varlen(g["q_nope"], g["q_pe"], g["k_nope"],
+                                                  g["k_pe"], g["v"], vl,
+                                                  softmax_scale=g["softmax_scale"]).cpu()
+    if mask is not None:
+        outs[tag + "m"] = binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"],
+                                               g["v"], mask=mask.to(dev),
+                                               softmax_scale=g["softmax_scale"]).cpu()
+
+for B, T in CASES:
+    run(inputs.make_inputs(B, T, seed=1300 + T + B, with_weight=False), f"r{B}x{T}", LENS(B, T))
+for B, T in PEAKED:
+    run(inputs.make_peaked_inputs(B, T, seed=1400 + T + B), f"p{B}x{T}", LENS(B, T))
+if MASK_FORMS:
+    for B, T in [(1, 256), (2, 300)]:
+        lens = [T] * B
+        run(inputs.make_inputs(B, T, seed=31 + T, with_weight=False), f"c{B}x{T}", lens,
+            inputs.keypad_mask(torch.tensor(lens), T))
+    lens = [700, 333, 129]
+    run(inputs.make_inputs(3, 700, seed=5, with_weight=False), "k3x700", lens,
+        inputs.keypad_mask(torch.tensor(lens), 700))
 torch.cuda.synchronize()
 st, word = binding.device_status()
 assert st == 0, (st, word)
 torch.save(outs, OUT)
 """
 
+LENS_SRC = "def LENS(B, T):\n    return [max(1, T - 77 * (b + 1)) for b in range(B)]\n"
 
-def run_child(kernel, out_path):
-    env = dict(os.environ, MLA_ATTN_KERNEL=kernel)
-    code = f"ROOT = {ROOT!r}\nOUT = {out_path!r}\nCASES = {CASES!r}\n" + CHILD
+
+def run_child(kernel, out_path, mask_forms=False):
+    env = dict(os.environ)
+    env.pop("MLA_ATTN_KERNEL", None)
+    if kernel != "half":
+        env["MLA_ATTN_KERNEL"] = kernel
+    code = (f"ROOT = {ROOT!r}\nOUT = {out_path!r}\nCASES = {CASES!r}\nPEAKED = {PEAKED!r}\n"
+            f"MASK_FORMS = {mask_forms!r}\n" + LENS_SRC + CHILD)
     res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
-                         timeout=600)
+                         timeout=900)
     assert res.returncode == 0, res.stderr[-3000:]
     return torch.load(out_path)
 
 
-def test_one_sm_and_pair_kernels_agree(cuda_device, tmp_path):
-    pair_all = run_child("pair", str(tmp_path / "pair.pt"))
-    one_sm = run_child("one_sm", str(tmp_path / "one_sm.pt"))
+def varlen_mask(B, T, lens):
+    return inputs.keypad_mask(torch.tensor(lens), T)
+
+
+def ulps(a, b):
+    """|a - b| in units of b's bf16 ulp, elementwise."""
+    diff = (a.float() - b.float()).abs()
+    return diff / (b.float().abs().clamp_min(1e-30).log2().floor() - 7).exp2()
+
+
+def oracle_case(d, mask):
+    ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], mask,
+                               d["softmax_scale"])
+    assert not fm.any()
+    return ref
+
+
+def test_kernels_against_oracle_and_each_other(cuda_device, tmp_path):
+    outs = {k: run_child(k, str(tmp_path / f"{k}.pt")) for k in ("half", "tile", "pair")}
     report = {}
-    for B, T in CASES:
-        d = inputs.make_inputs(B, T, seed=1300 + T + B, with_weight=False)
-        pair, pair_v = pair_all[f"{B}x{T}"], pair_all[f"{B}x{T}v"]
-        ref, _ = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], None,
-                                  d["softmax_scale"])
-        for name, got in (("pair", pair), ("one_sm", one_sm[f"{B}x{T}"])):
-            assert_parity(to_f64(got).reshape(B * T, -1), ref, f"{name} causal B={B} T={T}")
-        for a, b_, tag in ((pair, one_sm[f"{B}x{T}"], ""), (pair_v, one_sm[f"{B}x{T}v"], "v")):
-            diff = (a.float() - b_.float()).abs()
-            ulp = (b_.float().abs().clamp_min(1e-30).log2().floor() - 7).exp2()
-            report[f"{B}x{T}{tag}"] = {"equal": bool(torch.equal(a, b_)),
-                                       "max_diff_ulps": float((diff / ulp).max())}
-            assert float((diff / ulp).max()) <= 1.0, (B, T, tag, report)
+    err2 = {"half": 0.0, "tile": 0.0}
+    for kind, cases in (("r", CASES), ("p", PEAKED)):
+        for B, T in cases:
+            if kind == "r":
+                d = inputs.make_inputs(B, T, seed=1300 + T + B, with_weight=False)
+            else:
+                d = inputs.make_peaked_inputs(B, T, seed=1400 + T + B)
+            lens = lens_of(B, T)
+            for form, mask in (("", None), ("v", varlen_mask(B, T, lens))):
+                tag = f"{kind}{B}x{T}{form}"
+                ref = oracle_case(d, mask)
+                got = {k: to_f64(outs[k][tag]).reshape(B * T, -1) for k in outs}
+                for k in outs:
+                    assert_parity(got[k], ref, f"{k} {tag}")
+                if kind == "p":
+                    # rows with one answer: every row of the causal form; rows
+                    # t < len of the valid-length form
+                    rows = np.array([b * T + t for b in range(B) for t in range(T)
+                                     if form == "" or t < lens[b]])
+                    for k in outs:
+                        assert_peaked(got[k], ref, rows, f"{k} {tag}")
+                    continue
+                u = ulps(outs["pair"][tag], outs["tile"][tag])
+                report[tag] = {"pair_vs_tile_max_ulps": float(u.max())}
+                assert float(u.max()) <= 1.0, (tag, report)
+                # half vs tile: rows t < 64 see keys 0..63 only
+                first = [b * T + t for b in range(B) for t in range(min(T, 64))]
+                a = outs["half"][tag].reshape(B * T, -1)[first]
+                b_ = outs["tile"][tag].reshape(B * T, -1)[first]
+                assert torch.equal(a, b_), (tag, "rows t < 64 differ")
+                for k in err2:
+                    err2[k] += float(((got[k] - ref) ** 2).sum())
+                report[tag]["half_equal_tile"] = bool(torch.equal(outs["half"][tag],
+                                                                  outs["tile"][tag]))
+    rms = {k: v ** 0.5 for k, v in err2.items()}
+    report["err_norm"] = rms
     print(json.dumps(report))
+    assert rms["half"] <= 1.25 * rms["tile"] + 1e-9, report
+
+
+def test_tile_mode_mask_forms_are_bit_exact(cuda_device, tmp_path):
+    """On 128-key tiles: explicit causal mask == causal call; dense causal
+    key-padding mask == valid_len call outside the query tile holding the last
+    valid key."""
+    outs = run_child("tile", str(tmp_path / "tile.pt"), mask_forms=True)
+    for B, T in [(1, 256), (2, 300)]:
+        assert torch.equal(outs[f"c{B}x{T}m"], outs[f"c{B}x{T}"]), (B, T)
+    dense, compact = outs["k3x700m"], outs["k3x700v"]
+    T = 700
+    for b, L in enumerate([700, 333, 129]):
+        keep = torch.ones(T, dtype=torch.bool)
+        qt = (L - 1) // 128
+        if L < T:
+            keep[qt * 128:(qt + 1) * 128] = False
+        assert torch.equal(dense[b][keep], compact[b][keep]), f"b={b} L={L}"
