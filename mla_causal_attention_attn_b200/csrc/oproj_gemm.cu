@@ -4,9 +4,9 @@
 // page's parameter table gives W 8,192 x 7,168).
 //
 // Design (sm_100a):
-//   * persistent CTAs, one per SM, walking 128 x BN output tiles in a
-//     row-block-grouped order so concurrently running CTAs share A and W tiles
-//     in L2;
+//   * persistent CTAs, one per SM, walking MT*128 x BN output tiles in a
+//     grouped order (row groups for 128-row tiles, column groups for 256-row
+//     ones) so concurrently running CTAs share A and W tiles in L2;
 //   * warp 0 issues TMA loads of 128x64 A and BNx64 W tiles (128-byte
 //     swizzle) into a STAGES-deep shared-memory ring;
 //   * warp 1 allocates tensor memory and one elected thread issues
@@ -26,23 +26,41 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-// Output tiles are visited in groups of kGroupM row blocks (all column
-// blocks of a group before the next), so the tiles in flight share A rows and
-// W_o columns in L2. Groups of 8, 16 and 32 ran at the same speed on B200
-// (M = 4096 .. 32768, interleaved timing); 16 moved the least DRAM data.
+// Output tiles are visited in groups, so the tiles in flight share A rows
+// and W_o columns in L2. 128-row tiles: groups of kGroupM row blocks, all
+// column blocks of a group before the next (A band resident, W_o streamed);
+// groups of 8, 16 and 32 ran at the same speed (M = 4096 .. 32768), 16 moved
+// the least DRAM data. 256-row tiles: groups of kGroupN column blocks, all
+// row blocks of a group before the next (W_o band resident, A streamed):
+// measured against row groups at M = 16384 (ncu, one launch) 1.66 against
+// 1.84 GB of DRAM traffic, and 1-9 % less time at M = 16384 and 32768; at M
+// = 4096 (128-row tiles) column groups moved more data (540-617 against 462
+// MB) and were not faster.
 constexpr int kGroupM = 16;
+constexpr int kGroupN = 16;
 constexpr int kThreads = 192;
 constexpr int64_t kSmallMMax = 128;  // M up to this goes to oproj_small_m_kernel
 
+template <int MT>
 __device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_tiles, int& mb,
                                                  int& nb) {
-  const int group_tiles = kGroupM * n_tiles;
-  const int group = tile / group_tiles;
-  const int first_m = group * kGroupM;
-  const int gm = min(kGroupM, m_tiles - first_m);
-  const int in_group = tile - group * group_tiles;
-  mb = first_m + in_group % gm;
-  nb = in_group / gm;
+  if (MT == 1) {
+    const int group_tiles = kGroupM * n_tiles;
+    const int group = tile / group_tiles;
+    const int first_m = group * kGroupM;
+    const int gm = min(kGroupM, m_tiles - first_m);
+    const int in_group = tile - group * group_tiles;
+    mb = first_m + in_group % gm;
+    nb = in_group / gm;
+  } else {
+    const int group_tiles = kGroupN * m_tiles;
+    const int group = tile / group_tiles;
+    const int first_n = group * kGroupN;
+    const int gn = min(kGroupN, n_tiles - first_n);
+    const int in_group = tile - group * group_tiles;
+    nb = first_n + in_group % gn;
+    mb = in_group / gn;
+  }
 }
 
 // An output tile is MT x 128 rows by BN columns. MT = 1: two accumulators in
@@ -141,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         int mb, nb;
-        gemm_tile_coords(tile, m_tiles, n_tiles, mb, nb);
+        gemm_tile_coords<MT>(tile, m_tiles, n_tiles, mb, nb);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, ctl, 1)) {
             ok = false;
@@ -228,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       int mb, nb;
-      gemm_tile_coords(tile, m_tiles, n_tiles, mb, nb);
+      gemm_tile_coords<MT>(tile, m_tiles, n_tiles, mb, nb);
       const int buf = acc_buf(local);
       const uint32_t acc_par = acc_phase(local);
       if (!mbar_wait_warp(&acc_full[buf], acc_par, ctl, 6)) break;
