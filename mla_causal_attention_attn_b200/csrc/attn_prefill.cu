@@ -78,6 +78,7 @@ constexpr uint32_t kRegsControl = 88;
 constexpr uint32_t kRegsSoftmax = 208;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 384 * 168, "register split");
 constexpr int kBarTeardown = 1;  // named barrier for the final hand-off
+constexpr int kBarStage0 = 2;    // + query tile: its output rows are staged
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -421,7 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmQp,
                             const __grid_constant__ CUtensorMap tmKn,
                             const __grid_constant__ CUtensorMap tmKp,
-                            const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
+                            const __grid_constant__ CUtensorMap tmV,
+                            const __grid_constant__ CUtensorMap tmOut, const AttnArgs args) {
   static_assert(!(kMasked && kHalf), "half-tile scores serve the causal kernel only");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[2];     // query tile i is in shared memory
@@ -472,6 +474,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   WaitCtl ctl{&abort_flag, args.wait_limit_ns, kErrKernelAttn, args.err_word};
 
+  // TMA loads (thread 0, the producer): query tile i (nope lo, nope hi, rope:
+  // 48 KB), and block i of key tile k0 into ring slot `slot`.
+  auto load_q = [&](uint32_t i) {
+    uint8_t* sQ = smem + kOffQ + i * kQBytes;
+    const int q0 = tiles.qt[i] * kBQ;
+    mbar_arrive_expect_tx(&q_full[i], kQBytes);
+    tma_load_3d(sQ, &tmQn, &q_full[i], 0, q0, bh);
+    tma_load_3d(sQ + kBlock, &tmQn, &q_full[i], 64, q0, bh);
+    tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full[i], 0, q0, bh);
+  };
+  auto load_block = [&](int i, uint32_t slot, int k0) {
+    uint8_t* dst = smem + kOffRing + slot * kBlock;
+    mbar_arrive_expect_tx(&ring_full[slot], kBlock);
+    switch (i) {
+      case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0, bh); break;
+      case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0, bh); break;
+      case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0, b); break;
+      default: {
+        // V for 64 keys, all 128 value dims: two 64 x 64 boxes, 8 KB apart
+        const int kv = k0 + (i - 3) * 64;
+        tma_load_3d(dst, &tmV, &ring_full[slot], 0, kv, bh);
+        tma_load_3d(dst + kBlock / 2, &tmV, &ring_full[slot], 64, kv, bh);
+        break;
+      }
+    }
+  };
+  // The first key tile's K blocks (ring slots 0..2) and query tile 0 are
+  // loaded as soon as the barriers exist, overlapping the tensor-memory
+  // allocation and the block-wide barrier; the producer loop skips them.
+  constexpr uint32_t kPreBlocks = 3;
+
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(&q_full[0], 1);
@@ -495,6 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&never_bar, 1);
     }
     fence_barrier_init();
+    if (has_work) {
+      load_q(0);
+      for (uint32_t i = 0; i < kPreBlocks; ++i) load_block(int(i), i, tiles.first() * kBKV);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&tmem_slot, kTmemCols);
@@ -517,17 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tensormap(&tmKn);
       prefetch_tensormap(&tmKp);
       prefetch_tensormap(&tmV);
-      // Query tile 0, then the first key tile's K blocks, then query tile 1:
-      // the first S MMA waits for 96 KB rather than 144 KB.
-      auto load_q = [&](uint32_t i) {
-        uint8_t* sQ = smem + kOffQ + i * kQBytes;
-        const int q0 = tiles.qt[i] * kBQ;
-        mbar_arrive_expect_tx(&q_full[i], kQBytes);
-        tma_load_3d(sQ, &tmQn, &q_full[i], 0, q0, bh);
-        tma_load_3d(sQ + kBlock, &tmQn, &q_full[i], 64, q0, bh);
-        tma_load_3d(sQ + 2 * kBlock, &tmQp, &q_full[i], 0, q0, bh);
-      };
-      load_q(0);
+      // Query tile 0 and the first key tile's K blocks came with the
+      // barriers; query tile 1 follows them, so the first S MMA waits for
+      // 96 KB rather than 144 KB.
       bool q1_issued = false;
       uint32_t issued = 0, issued_par = 0;
       uint32_t s = 0;  // block sequence number
@@ -558,20 +587,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBlocksPerTile; ++i, ++s) {
           const uint32_t slot = s % kRing;
           const uint32_t par = (s / kRing) & 1u;
-          if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
-          uint8_t* dst = smem + kOffRing + slot * kBlock;
-          mbar_arrive_expect_tx(&ring_full[slot], kBlock);
-          switch (i) {
-            case 0: tma_load_3d(dst, &tmKn, &ring_full[slot], 0, k0, bh); break;
-            case 1: tma_load_3d(dst, &tmKn, &ring_full[slot], 64, k0, bh); break;
-            case 2: tma_load_3d(dst, &tmKp, &ring_full[slot], 0, k0, b); break;
-            default: {
-              // V for 64 keys, all 128 value dims: two 64 x 64 boxes, 8 KB apart
-              const int kv = k0 + (i - 3) * 64;
-              tma_load_3d(dst, &tmV, &ring_full[slot], 0, kv, bh);
-              tma_load_3d(dst + kBlock / 2, &tmV, &ring_full[slot], 64, kv, bh);
-              break;
-            }
+          if (s >= kPreBlocks) {
+            if (!mbar_wait(&ring_empty[slot], par ^ 1u, ctl, 1)) { ok = false; break; }
+            load_block(i, slot, k0);
           }
           issued |= 1u << slot;
           issued_par = (issued_par & ~(1u << slot)) | (par << slot);
@@ -942,12 +960,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]
-    const bool have = ok && n > 0 && mbar_wait_warp(&o_final[wi], 0, ctl, 22);
-    if (have) tc_fence_after();
-    if (n == 0 || have) {
+    // epilogue: O / l -> bf16 -> out[b, q, h*128 + e]. The rows are staged
+    // in this query tile's Q buffer (free: its last S product has completed)
+    // as two 128-row x 64-dim boxes in the TMA 128-byte swizzle (16-byte
+    // chunk c of row r at chunk c ^ (r % 8), so the warp's stores spread
+    // over all banks), then written by two TMA stores. Rows at or past T
+    // fall outside the output map's T extent and are not written.
+    // A query tile with no key tiles to visit writes zeros; its buffer may
+    // still be receiving its query rows, which land first. Every warp of the
+    // warpgroup reaches the staging barrier whatever happened before it; the
+    // rows are stored only if all four staged theirs.
+    bool stage_ok = false;
+    if (ok && n > 0) {
+      stage_ok = mbar_wait_warp(&o_final[wi], 0, ctl, 22);
+      if (stage_ok) tc_fence_after();
+    } else if (ok) {
+      stage_ok = !(has_work && tiles.exists[wi]) || mbar_wait_warp(&q_full[wi], 0, ctl, 25);
+    }
+    uint8_t* stage = smem + kOffQ + wi * kQBytes;
+    if (stage_ok) {
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = args.out + (size_t(b) * args.T + q) * size_t(kH * kDV) + h * kDV;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t rr[32];
@@ -964,14 +996,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i)
           packed[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l,
                                   __uint_as_float(rr[2 * i + 1]) * inv_l);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        // dims 32c .. 32c+31: box c / 2, 16-byte chunks 4 (c % 2) .. + 3
+        uint8_t* rowp = stage + (c >> 1) * kBlock + r * 128;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
-                                packed[4 * i + 3]);
+        for (int i = 0; i < 4; ++i) {
+          const int chunk = 4 * (c & 1) + i;
+          *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
       }
+      fence_proxy_async_smem();
+    }
+    const bool all_staged = named_barrier_and(kBarStage0 + wi, 128, stage_ok);
+    if (all_staged && tiles.exists[wi] && quad == 0 && lane == 0) {
+      tma_store_3d(&tmOut, stage, h * kDV, qt * kBQ, b);
+      tma_store_3d(&tmOut, stage + kBlock, h * kDV + 64, qt * kBQ, b);
+      bulk_commit_group();
+      bulk_wait_group_read<0>();  // the staging buffer stays valid until read
     }
   }
 
@@ -1841,9 +1882,10 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                                                   a);
     return cudaGetLastError();
   }
+  CUtensorMap tmOut;  // out [B, T, 64 * 128]: 64-dim x 128-row boxes
   if (!make_map_3d(&tmQn, q_nope, kDN, T, BH) || !make_map_3d(&tmQp, q_pe, kDR, T, BH) ||
       !make_map_3d(&tmKn, k_nope, kDN, T, BH) || !make_map_3d(&tmKp, k_pe, kDR, T, B) ||
-      !make_map_3d(&tmV, v, kDV, T, BH, 64))
+      !make_map_3d(&tmV, v, kDV, T, BH, 64) || !make_map_3d(&tmOut, out, kH * kDV, T, B))
     return cudaErrorInvalidValue;
   // causal and valid-length calls: half-tile scores unless MLA_ATTN_KERNEL=tile
   const bool half = !mask && !tile_kernel_selected();
@@ -1876,7 +1918,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
   a.rope_cs = static_cast<const float2*>(rope_cs);
   const long long ctas = (long long)B * kH * a.n_pairs;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidValue;
-  kern<<<unsigned(ctas), kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, a);
+  kern<<<unsigned(ctas), kThreads, kSmemBytes, stream>>>(tmQn, tmQp, tmKn, tmKp, tmV, tmOut, a);
   return cudaGetLastError();
 }
 
