@@ -1895,7 +1895,7 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
                                     : mla_attn_prefill_kernel<false, false, true>)
                          : (rope_cs ? mla_attn_prefill_kernel<false, true, false>
                                     : mla_attn_prefill_kernel<false, false, false>);
-  static ContextCache attr_done[6];
+  static ContextCache attr_done[8];  // index: mask + 2 rope + 4 half
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemBytes),
                                    &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0) + (half ? 4 : 0)]);
   if (e != cudaSuccess) return e;

@@ -39,6 +39,7 @@
 #include <cuda_fp8.h>
 
 #include "../../include/mla.h"
+#include "fp8_codes.cuh"
 #include "host_util.h"
 #include "sm100.cuh"
 
@@ -47,20 +48,9 @@ namespace mla {
 namespace {
 
 constexpr int kGroup = 128;        // quantisation group along K, and weight block edge
-constexpr float kE4m3Max = 448.f;  // largest finite e4m3 value
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ float group_scale(float amax) {
-  return amax > 0.f ? __fdiv_rn(amax, kE4m3Max) : 1.f;
-}
-
-// e4m3 code of x / s: fp32 quotient rounded to nearest, then the nearest
-// e4m3 value (ties to even), saturating at +-448.
-__device__ __forceinline__ uint32_t e4m3_code(float x, float s) {
-  return uint32_t(__nv_cvt_float_to_fp8(__fdiv_rn(x, s), __NV_SATFINITE, __NV_E4M3));
-}
 
 // ---------------------------------------------------------------- quantisers
 // x [M, K] bf16 (row stride ld elements) -> q [M, K] codes, scale [K/128][M].
@@ -176,8 +166,16 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- GEMM
 constexpr int kBM = 128;
-constexpr int kPromoWarps = 8;       // warps 2..9: two sets of four, BN/2 columns each
-constexpr int kThreads = 64 + 32 * kPromoWarps;
+// Warpgroup 0: TMA producer (warp 0), tensor-memory owner and MMA issuer
+// (warp 1), two idle warps. Warpgroups 1 and 2: the promotion warps 4..11, two
+// sets of four, BN/2 columns each. The roles are warpgroup-aligned so that
+// setmaxnreg can move registers to the promotion warps (BN = 256 holds 128
+// fp32 accumulators a thread): 128 x 72 + 256 x 216 = 384 x 168.
+constexpr int kPromoWarps = 8;
+constexpr int kThreads = 128 + 32 * kPromoWarps;
+constexpr uint32_t kRegsCtl = 72;
+constexpr uint32_t kRegsPromo = 216;
+static_assert(128 * kRegsCtl + 32 * kPromoWarps * kRegsPromo <= kThreads * 168, "register split");
 constexpr uint32_t kABytes = kBM * kGroup;
 constexpr int kGroupM = 16;          // row blocks visited together (L2 reuse)
 constexpr int kScaleAhead = 4;       // groups of scales loaded ahead
@@ -264,6 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtl>();
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -349,11 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&drain_bar, 0, drain, 5);
       }
     }
+  }
   } else {
+    setmaxnreg_inc<kRegsPromo>();
     // ---------------------------------------------------------------- promotion + epilogue
     constexpr int kCols = Cfg::kCols, kChunk = Cfg::kChunk;
     const int quad = warp & 3;                     // TMEM lane quadrant this warp may access
-    const int col0 = ((warp - 2) >> 2) * kCols;    // this warp's columns of the tile
+    const int col0 = ((warp - 4) >> 2) * kCols;    // this warp's columns of the tile
     const int row_in_tile = quad * 32 + lane;
     int part = 0;
     uint32_t part_phase = 0;
