@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from mla_causal_attention_attn_b200 import binding, inputs
-from parity import assert_parity, sample_rows, to_f64
+from parity import assert_parity, assert_peaked, sample_rows, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -108,3 +108,38 @@ def test_varlen_fused_full_size_sampled_rows(cuda_device):
     assert not fm.any()
     m = assert_parity(got, ref, f"varlen fused b8_t4096 ({len(rows)} rows)")
     print(m)
+
+
+@pytest.mark.parametrize("B,T,lens", [
+    (6, 320, [63, 64, 65, 127, 128, 129]),   # key limits on both sides of 64-key halves
+    (4, 191, [191, 190, 192, 1]),            # ragged T inside a second half tile
+    (3, 257, [257, 193, 2]),                 # one row past two full tiles
+])
+def test_varlen_half_tile_boundaries_peaked(cuda_device, B, T, lens):
+    """Causal attention scores 64 keys at a time. On inputs whose query row i
+    points at keys i and i+1, every row t < len(b) has the answer v_t,
+    checked element by element within half a bf16 ulp, so a key limit that
+    is off by one at a 64-key boundary, a ragged tail or the diagonal fails
+    here. Rows t >= len(b) match the oracle under the path's tolerance."""
+    d = inputs.make_peaked_inputs(B, T, seed=B * 31 + T)
+    vl = torch.tensor(lens, dtype=torch.int32)
+    clamped = vl.clamp(0, T).to(torch.int64)
+    mask = inputs.keypad_mask(clamped, T)
+    ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], mask,
+                               d["softmax_scale"])
+    assert not fm.any()
+    g = to_dev(d, cuda_device)
+    out = gpu_varlen(g, vl.to(cuda_device))
+    causal = binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                                  softmax_scale=g["softmax_scale"])
+    torch.cuda.synchronize()
+    check_status()
+    got = to_f64(out).reshape(B * T, -1)
+    assert_parity(got, ref, f"varlen peaked B={B} T={T}")
+    rows = np.array([b * T + t for b in range(B) for t in range(int(clamped[b]))])
+    assert_peaked(got, ref, rows, f"varlen peaked B={B} T={T}")
+    # plain causal on the same inputs: every row has one answer
+    ref_c, _ = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"], None,
+                                d["softmax_scale"])
+    got_c = to_f64(causal).reshape(B * T, -1)
+    assert_peaked(got_c, ref_c, np.arange(B * T), f"causal peaked B={B} T={T}")
