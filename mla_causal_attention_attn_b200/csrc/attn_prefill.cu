@@ -68,7 +68,12 @@ constexpr int kDN = 128;     // qk_nope_head_dim
 constexpr int kDR = 64;      // qk_rope_head_dim
 constexpr int kDV = 128;     // v_head_dim
 constexpr int kH = 64;       // heads
-constexpr int kHeadGroup = 8;  // heads whose CTAs are scheduled together (L2 reuse of K/V)
+// Heads whose CTAs are scheduled together (L2 reuse of K/V): 8 (a group's
+// K/V of 8 x 2 MB at T = 4096 stays in L2), more for short sequences, where
+// a group's K/V is small and a longer longest-first run packs the SMs
+// better.
+constexpr int kHeadGroup = 8;
+__host__ __device__ constexpr int head_group_for(int T) { return T <= 2048 ? 16 : kHeadGroup; }
 constexpr int kRing = 8;     // 16 KB blocks in the K/V ring
 constexpr int kBlocksPerTile = 5;
 constexpr int kThreads = 384;
@@ -446,14 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // CTA -> (b, h, pair): groups of kHeadGroup heads, longest pairs first
+  // CTA -> (b, h, pair): groups of head_group_for(T) heads, longest pairs first
   // within a group.
-  const int per_group = kHeadGroup * args.n_pairs;
+  const int hg = head_group_for(args.T);
+  const int per_group = hg * args.n_pairs;
   const int grp = blockIdx.x / per_group;
   const int rem = blockIdx.x - grp * per_group;
-  const int b = grp / (kH / kHeadGroup);
-  const int h = (grp % (kH / kHeadGroup)) * kHeadGroup + rem % kHeadGroup;
-  const int pair = args.n_pairs - 1 - rem / kHeadGroup;
+  const int b = grp / (kH / hg);
+  const int h = (grp % (kH / hg)) * hg + rem % hg;
+  const int pair = args.n_pairs - 1 - rem / hg;
   const int bh = b * kH + h;
   // Keys of this sequence: T, or valid_len[b] clamped to [0, T].
   const int n_keys =
