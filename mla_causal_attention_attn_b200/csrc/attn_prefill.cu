@@ -17,8 +17,9 @@
 // every K/V tile brought into shared memory serves 256 query rows and the
 // softmax of one query tile overlaps the tensor-core work of the other.
 // Roles (384 threads = three warpgroups):
-//   warp 0       TMA producer: query tile 0 (nope + rope, 48 KB), the first key
-//                tile's K blocks, query tile 1, then for every visited 128-key
+//   warp 0       TMA producer: query tile 0 (nope + rope, 48 KB) and the first
+//                key tile's K blocks (issued by thread 0 right after it sets up
+//                the barriers), query tile 1, then for every visited 128-key
 //                tile five 16 KB blocks (k_nope lo/hi, the shared k_pe,
 //                v lo/hi) into an 8-block ring;
 //   warp 1       tensor-memory owner; warps 1 and 2: one MMA-issuing thread
@@ -35,7 +36,8 @@
 //   warps 8..11  softmax of query tile 1. Each reads S, scales, masks, keeps a
 //                running max (rescaling O only when the max grows by more than
 //                2^8), exponentiates, sums, writes P as bf16 over the first 64
-//                columns of its S buffer, and at the end O / l -> bf16 -> out.
+//                columns of its S buffer, and at the end O / l -> bf16, staged in
+//                its query tile's freed Q buffer and written by TMA stores.
 //                Tiles that need no mask entries added (every causal tile, the
 //                all-zero tiles of an explicit mask) take a single pass
 //                against the running max; the others two passes.
