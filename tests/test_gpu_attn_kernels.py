@@ -79,22 +79,66 @@ if MASK_FORMS:
     lens = [700, 333, 129]
     run(inputs.make_inputs(3, 700, seed=5, with_weight=False), "k3x700", lens,
         inputs.keypad_mask(torch.tensor(lens), 700))
+if EXTRA:
+    # explicit masks (a general additive one, a causal key-padding one) and
+    # the rotary call, with and without a mask: these run the selected
+    # kernel's masked and rotary instances
+    for tag, d in EXTRA_INPUTS().items():
+        g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+        m = g["mask"]
+        if tag.startswith("rope"):
+            outs[tag] = binding.attn_prefill_rope(
+                g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"], g["v"],
+                position_ids=g["pos"], rope=inputs.KIMI_K2_ROPE, mask=m,
+                softmax_scale=g["softmax_scale"]).cpu()
+        else:
+            outs[tag] = binding.attn_prefill(g["q_nope"], g["q_pe"], g["k_nope"], g["k_pe"],
+                                             g["v"], mask=m,
+                                             softmax_scale=g["softmax_scale"]).cpu()
 torch.cuda.synchronize()
 st, word = binding.device_status()
 assert st == 0, (st, word)
 torch.save(outs, OUT)
 """
 
+EXTRA_SRC = r"""
+def EXTRA_INPUTS():
+    import torch
+    from mla_causal_attention_attn_b200 import inputs
+    out = {}
+    d = inputs.make_inputs(2, 300, seed=901, with_weight=False)
+    gm = torch.Generator().manual_seed(902)
+    m = torch.randn(2, 1, 300, 300, generator=gm) * 2.0
+    m.masked_fill_(torch.rand(2, 1, 300, 300, generator=gm) < 0.3, float("-inf"))
+    m[..., 0] = 0.0
+    d["mask"] = m.to(torch.bfloat16)
+    out["gen2x300"] = d
+    d = inputs.make_inputs(2, 300, seed=903, with_weight=False)
+    d["mask"] = inputs.keypad_mask(torch.tensor([300, 150]), 300)
+    out["kp2x300"] = d
+    d = inputs.make_inputs(2, 300, seed=904, with_weight=False)
+    d["pos"] = inputs.make_positions(2, 300, "offset")
+    out["rope2x300"] = d
+    d = dict(inputs.make_inputs(2, 300, seed=905, with_weight=False))
+    d["pos"] = inputs.make_positions(2, 300, "random", seed=906)
+    d["mask"] = inputs.keypad_mask(torch.tensor([300, 111]), 300)
+    out["ropem2x300"] = d
+    return out
+"""
+exec(EXTRA_SRC)
+
 LENS_SRC = "def LENS(B, T):\n    return [max(1, T - 77 * (b + 1)) for b in range(B)]\n"
 
 
-def run_child(kernel, out_path, mask_forms=False):
+def run_child(kernel, out_path, mask_forms=False, extra=False, cases=None, peaked=None):
     env = dict(os.environ)
     env.pop("MLA_ATTN_KERNEL", None)
     if kernel != "half":
         env["MLA_ATTN_KERNEL"] = kernel
-    code = (f"ROOT = {ROOT!r}\nOUT = {out_path!r}\nCASES = {CASES!r}\nPEAKED = {PEAKED!r}\n"
-            f"MASK_FORMS = {mask_forms!r}\n" + LENS_SRC + CHILD)
+    cases = CASES if cases is None else cases
+    peaked = PEAKED if peaked is None else peaked
+    code = (f"ROOT = {ROOT!r}\nOUT = {out_path!r}\nCASES = {cases!r}\nPEAKED = {peaked!r}\n"
+            f"MASK_FORMS = {mask_forms!r}\nEXTRA = {extra!r}\n" + LENS_SRC + EXTRA_SRC + CHILD)
     res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
                          timeout=900)
     assert res.returncode == 0, res.stderr[-3000:]
@@ -176,3 +220,29 @@ def test_tile_mode_mask_forms_are_bit_exact(cuda_device, tmp_path):
         if L < T:
             keep[qt * 128:(qt + 1) * 128] = False
         assert torch.equal(dense[b][keep], compact[b][keep]), f"b={b} L={L}"
+
+
+def test_every_kernel_masks_and_rotary_against_oracle(cuda_device, tmp_path):
+    """The explicit-mask and rotary instances of each kernel setting (the
+    CTA-pair kernel runs them too when selected) against the fp64 oracle: a
+    general additive mask, a causal key-padding mask, and the rotary call
+    with offset positions, and with random positions under a mask."""
+    want = {}
+    for tag, d in EXTRA_INPUTS().items():
+        B, _, T, _ = d["q_nope"].shape
+        if tag.startswith("rope"):
+            ref, fm = oracle.attn_rows_rope(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"],
+                                            d["v"], d["mask"], d["softmax_scale"], d["pos"],
+                                            inputs.KIMI_K2_ROPE)
+        else:
+            ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                                       d["mask"], d["softmax_scale"])
+        want[tag] = (ref, fm, B, T)
+    for kernel in ("half", "tile", "pair"):
+        outs = run_child(kernel, str(tmp_path / f"x_{kernel}.pt"), extra=True, cases=[],
+                         peaked=[])
+        for tag, (ref, fm, B, T) in want.items():
+            got = to_f64(outs[tag]).reshape(B * T, -1)
+            rows = ~fm.any(axis=1)
+            assert np.all(got[~rows] == 0.0), (kernel, tag)
+            assert_parity(got[rows], ref[rows], f"{kernel} {tag}")
