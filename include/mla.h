@@ -45,6 +45,14 @@
  *    streams report into the same word) and the no-alloc call's fixed
  *    scratch. Cached per device and context: the SM count, device addresses
  *    of the library's module variables, kernel attributes.
+ *  - Environment (each read once per process): MLA_WAIT_LIMIT_NS sets the
+ *    bounded waits' limit in nanoseconds; MLA_ATTN_KERNEL selects the
+ *    attention kernel: unset, the one-SM kernel with 64-key score halves for
+ *    causal and valid-length calls (128-key tiles for explicit masks);
+ *    "tile", 128-key tiles for every call; "pair", the CTA-pair kernel for
+ *    every call. The choice changes rounding order only: every setting
+ *    meets the same tolerance. MLA_TEST_STALL_WAIT makes
+ *    one bounded wait never complete, for failure-detection tests.
  */
 #ifndef MLA_B200_H_
 #define MLA_B200_H_
