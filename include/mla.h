@@ -51,7 +51,10 @@
  *    causal and valid-length calls (128-key tiles for explicit masks);
  *    "tile", 128-key tiles for every call; "pair", the CTA-pair kernel for
  *    every call. The choice changes rounding order only: every setting
- *    meets the same tolerance. MLA_TEST_STALL_WAIT makes
+ *    meets the same tolerance. MLA_ATTN_PV_ISSUER ("1" or "0") overrides
+ *    which thread issues the 64-key halves' PV products (a thread of their
+ *    own from T = 4096 on, else each query tile's MMA issuer); both give
+ *    bit-identical results. MLA_TEST_STALL_WAIT makes
  *    one bounded wait never complete, for failure-detection tests.
  */
 #ifndef MLA_B200_H_

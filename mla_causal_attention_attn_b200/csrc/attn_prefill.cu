@@ -31,7 +31,8 @@
 //                S0_j, S1_j, S0_{j+1}, ... Because PV_{j-1} of a tile is issued
 //                before its S_j, the commit that announces S_j also guarantees
 //                O holds PV_{j-1};
-//   warp 3       idle;
+//   warp 3       idle, or (half-tile scores, long sequences) the PV issuer
+//                described below;
 //   warps 4..7   softmax of query tile 0, one thread per row (TMEM lane);
 //   warps 8..11  softmax of query tile 1. Each reads S, scales, masks, keeps a
 //                running max (rescaling O only when the max grows by more than
@@ -52,6 +53,15 @@
 // the softmax waits for PV(u-1) only before it rescales O. The O accumulators
 // and the K/V ring are unchanged. Explicit masks keep 128-key tiles (a query
 // tile there may skip key tiles in the middle of the visited ones).
+//
+// Separate PV issuer (half tiles, T >= kPvIssuerMinT unless MLA_ATTN_PV_ISSUER
+// says otherwise): an issuer that waits for a K block of S(u+2) cannot issue
+// PV(u+1), however early P(u+1) is written. Then warps 1 and 2 issue only the
+// S products, and one thread of warp 3 issues the PV products of both query
+// tiles, polling P and V readiness of each tile in turn. S(u+2) overwrites
+// the buffer PV(u) reads, so the S issuer waits until PV(u) has been issued
+// (pv_issued); the tensor pipe keeps that order across the two threads
+// through the tcgen05 fences around the barrier.
 #include "attn_prefill.h"
 
 #include <cstdlib>
@@ -77,6 +87,13 @@ constexpr int kH = 64;       // heads
 constexpr int kHeadGroup = 8;
 __host__ __device__ constexpr int head_group_for(int T) { return T <= 2048 ? 16 : kHeadGroup; }
 constexpr int kRing = 8;     // 16 KB blocks in the K/V ring
+// Sequences at least this long issue their half-tile PV products from a
+// thread of their own. Shorter ones keep one issuer per query tile: there
+// the last query tile runs alone for a larger share of a CTA, and the extra
+// hand-off between S and PV issuers sits on its serial chain (B=16 T=1024:
+// 0.549 against 0.516 ms; B=1 T=4096: 0.342 against 0.345 ms; B=1 T=32768:
+// 20.1-20.2 against 20.8-21.0 ms).
+constexpr int kPvIssuerMinT = 4096;
 constexpr int kBlocksPerTile = 5;
 constexpr int kThreads = 384;
 // ptxas budgets 168 registers a thread for 384 threads; setmaxnreg moves
@@ -423,7 +440,7 @@ __device__ __forceinline__ bool softmax_step(const AttnArgs& args, uint32_t lane
   return true;
 }
 
-template <bool kMasked, bool kRope, bool kHalf>
+template <bool kMasked, bool kRope, bool kHalf, bool kPvIssuer>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQn,
                             const __grid_constant__ CUtensorMap tmQp,
@@ -432,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmOut, const AttnArgs args) {
   static_assert(!(kMasked && kHalf), "half-tile scores serve the causal kernel only");
+  static_assert(kHalf || !kPvIssuer, "the PV issuer serves half-tile scores");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[2];     // query tile i is in shared memory
   __shared__ uint64_t q_rot[2];      // its rotary part is rotated (rotary calls only)
@@ -440,8 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // half] on half tiles
   __shared__ uint64_t s_full[4], p_full[4];
   __shared__ uint64_t pv_done[2];   // half tiles: a PV product of query tile i completed
+  // half tiles with a PV issuer: PV(u) of query tile i has been issued,
+  // [2 * i + u % 2]
+  __shared__ uint64_t pv_issued[4];
   __shared__ uint64_t o_final[2];
-  __shared__ uint64_t drain_bar[2];
+  __shared__ uint64_t drain_bar[3];  // issuer i's MMAs (i = 2: the PV issuer) have completed
   __shared__ uint64_t s_issued[2];  // issuer i has issued (or skipped) S of its next tile
   __shared__ uint64_t never_bar;    // no thread ever arrives (failure-detection test)
   __shared__ uint32_t tmem_slot;
@@ -521,16 +542,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&q_rot[1], 128);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&ring_full[s], 1);
-      // released once by each query tile's MMA issuer
+      // released once per query tile: K blocks by its S issuer, V blocks by
+      // its PV issuer (the same thread unless warp 3 issues the PVs)
       mbar_init(&ring_empty[s], tiles.exists[1] ? 2 : 1);
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      if (kPvIssuer) mbar_init(&pv_issued[i], 1);
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&drain_bar[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&o_final[i], 1);
-      mbar_init(&drain_bar[i], 1);
       mbar_init(&s_issued[i], 1);
       mbar_init(&pv_done[i], 1);
       mbar_init(&never_bar, 1);
@@ -713,11 +736,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         if (ok) ok = issue_s(0);
         if (ok) ok = issue_s(1);
-        for (int u = 0; ok && u < n_sub; ++u) {
-          ok = issue_pv(u);
-          if (ok && u + 2 < n_sub) ok = issue_s(u + 2);
+        if constexpr (kPvIssuer) {
+          // PV(u) comes from warp 3; S(u+2) follows it into the buffer.
+          (void)issue_pv;
+          for (int u = 0; ok && u + 2 < n_sub; ++u) {
+            ok = mbar_wait(&pv_issued[2 * qi + (u & 1)], uint32_t(u >> 1) & 1u, ctl, 18);
+            if (ok) {
+              tc_fence_after();
+              ok = issue_s(u + 2);
+            }
+          }
+        } else {
+          for (int u = 0; ok && u < n_sub; ++u) {
+            ok = issue_pv(u);
+            if (ok && u + 2 < n_sub) ok = issue_s(u + 2);
+          }
+          if (ok) mma_commit(&o_final[qi]);
         }
-        if (ok) mma_commit(&o_final[qi]);
         // The visited key tile past this query tile's last one (causal: the
         // other query tile's diagonal) is released unused, block by block
         // once it has landed, after every block this tile used.
@@ -810,6 +845,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         int zero = 0;
         WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
         mbar_wait(&drain_bar[qi], 0, drain, 14);
+      }
+    }
+  }
+  if constexpr (kPvIssuer) {
+    if (warp == 3 && lane == 0 && has_work) {
+      // ------------------------------------------------------------ PV issuer
+      // For each query tile in turn: once P(u) is written and the V block of
+      // half tile u has landed, O += P(u) V, release the V block, and tell
+      // the tile's S issuer (pv_issued). Spins on non-blocking tests: parking
+      // on one tile's barrier would hold up the other tile's PV. The tile
+      // loop stays rolled: unrolled, the tighter spin measured slower
+      // (B=1 T=32768: 20.5-20.6 against 19.8-19.9 ms), the thread sharing
+      // its SM sub-partition with two softmax warps.
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kBQ, kDV, false, true);
+      const uint32_t ring0 = smem_u32(smem + kOffRing);
+      int n_sub[2], next[2] = {0, 0};
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        n_sub[t] = tiles.exists[t] ? 2 * min(tiles.qt[t] + 1, tiles.end) : 0;
+      bool ok = true, issued_any = false;
+      unsigned long long last = globaltimer_ns();
+      while (ok && (next[0] < n_sub[0] || next[1] < n_sub[1])) {
+        bool progress = false;
+#pragma unroll 1
+        for (int t = 0; t < 2; ++t) {
+          const int u = next[t];
+          if (u >= n_sub[t]) continue;
+          const int kt = u >> 1, hb = u & 1;
+          const uint32_t vseq = kBlocksPerTile * uint32_t(kt) + 3 + hb;
+          if (!mbar_test(&p_full[2 * t + hb], uint32_t(u >> 1) & 1u) ||
+              !mbar_test(&ring_full[vseq % kRing], (vseq / kRing) & 1u))
+            continue;
+          tc_fence_after();
+          const uint32_t o_tmem = tmem_base + kColO + 128 * t;
+          const uint32_t p_tmem = tmem_base + kColS + 128 * t + 64 * hb;
+          const uint32_t vb = ring0 + (vseq % kRing) * kBlock;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
+            mma_ts(o_tmem, p_tmem + kk * 8, vd, idesc_o, (u | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&pv_done[t]);
+          mma_commit(&ring_empty[vseq % kRing]);
+          if (u + 1 == n_sub[t]) mma_commit(&o_final[t]);
+          tc_fence_before();
+          mbar_arrive(&pv_issued[2 * t + hb]);
+          issued_any = true;
+          next[t] = u + 1;
+          progress = true;
+        }
+        if (progress) {
+          last = globaltimer_ns();
+        } else if (abort_flag) {
+          ok = false;
+        } else if (globaltimer_ns() - last > args.wait_limit_ns) {
+          abort_flag = 1;
+          atomicCAS(args.err_word, 0u, kErrTimeoutFlag | kErrKernelAttn | 19u);
+          __threadfence();
+          ok = false;
+        }
+      }
+      if (!ok && issued_any) {
+        mma_commit(&drain_bar[2]);
+        int zero = 0;
+        WaitCtl drain{&zero, args.wait_limit_ns, kErrKernelAttn, args.err_word};
+        mbar_wait(&drain_bar[2], 0, drain, 14);
       }
     }
   }
@@ -1812,6 +1913,19 @@ bool tile_kernel_selected() {
   return v;
 }
 
+// Half-tile PV products from their own issuing thread: for T >=
+// kPvIssuerMinT, or as MLA_ATTN_PV_ISSUER (read once) says: "1" always,
+// "0" never.
+bool pv_issuer_for(int T) {
+  static const int env = [] {
+    const char* s = std::getenv("MLA_ATTN_PV_ISSUER");
+    if (s && std::strcmp(s, "1") == 0) return 1;
+    if (s && std::strcmp(s, "0") == 0) return 0;
+    return -1;
+  }();
+  return env >= 0 ? env == 1 : T >= kPvIssuerMinT;
+}
+
 // Rows of the mask can be read with 16-byte loads.
 bool mask_rows_vec_ok(const void* mask, int64_t mask_ld) {
   return (reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (mask_ld % 8) == 0;
@@ -1897,15 +2011,19 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
     return cudaErrorInvalidValue;
   // causal and valid-length calls: half-tile scores unless MLA_ATTN_KERNEL=tile
   const bool half = !mask && !tile_kernel_selected();
-  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, false>
-                             : mla_attn_prefill_kernel<true, false, false>)
-                  : half ? (rope_cs ? mla_attn_prefill_kernel<false, true, true>
-                                    : mla_attn_prefill_kernel<false, false, true>)
-                         : (rope_cs ? mla_attn_prefill_kernel<false, true, false>
-                                    : mla_attn_prefill_kernel<false, false, false>);
-  static ContextCache attr_done[8];  // index: mask + 2 rope + 4 half
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), int(kSmemBytes),
-                                   &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0) + (half ? 4 : 0)]);
+  const bool pv = half && pv_issuer_for(T);
+  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, false, false>
+                             : mla_attn_prefill_kernel<true, false, false, false>)
+              : pv ? (rope_cs ? mla_attn_prefill_kernel<false, true, true, true>
+                              : mla_attn_prefill_kernel<false, false, true, true>)
+              : half ? (rope_cs ? mla_attn_prefill_kernel<false, true, true, false>
+                                : mla_attn_prefill_kernel<false, false, true, false>)
+                     : (rope_cs ? mla_attn_prefill_kernel<false, true, false, false>
+                                : mla_attn_prefill_kernel<false, false, false, false>);
+  static ContextCache attr_done[16];  // index: mask + 2 rope + 4 half + 8 PV issuer
+  cudaError_t e = ensure_smem_attr(
+      reinterpret_cast<const void*>(kern), int(kSmemBytes),
+      &attr_done[(mask ? 1 : 0) + (rope_cs ? 2 : 0) + (half ? 4 : 0) + (pv ? 8 : 0)]);
   if (e != cudaSuccess) return e;
   AttnArgs a;
   a.mask = static_cast<const __nv_bfloat16*>(mask);

@@ -3,8 +3,11 @@
 Causal and valid-length calls run, by MLA_ATTN_KERNEL (read once per
 process), the one-SM kernel with 64-key (half-tile) score buffers (the
 default), the same kernel on 128-key tiles ("tile", the tiles explicit masks
-always use), or the CTA-pair kernel ("pair"). Each runs here in a child
-process with the variable set. Checked:
+always use), or the CTA-pair kernel ("pair"). The half-tile kernel issues
+its PV products either from each query tile's MMA issuer ("half") or from a
+thread of their own ("halfpv"; MLA_ATTN_PV_ISSUER=1, the default from
+T = 4096 on). Each runs here in a child process with the variables set.
+Checked:
 - every kernel against the fp64 oracle, on random inputs (causal and
   valid_len) and on inputs whose query row i points at keys i and i+1
   (inputs.make_peaked_inputs). On those the causal answer of row i is v_i to
@@ -12,6 +15,8 @@ process with the variable set. Checked:
   ulp: a kernel that let key i+1 in, or kept key i out, would be off by the
   size of v itself, at any row, tile boundary or ragged tail. The running
   max jumps on the diagonal there, so the rescale of O is exercised too;
+- the two half-tile issue orders run the same MMAs on the same operands in
+  the same order per accumulator: bit-identical outputs;
 - the tile and pair kernels do the same per-row arithmetic (128-key tiles,
   the same softmax routes): equal to within one bf16 ulp;
 - the half-tile kernel against the tile kernel: rows whose allowed keys all
@@ -133,7 +138,8 @@ LENS_SRC = "def LENS(B, T):\n    return [max(1, T - 77 * (b + 1)) for b in range
 def run_child(kernel, out_path, mask_forms=False, extra=False, cases=None, peaked=None):
     env = dict(os.environ)
     env.pop("MLA_ATTN_KERNEL", None)
-    if kernel != "half":
+    env["MLA_ATTN_PV_ISSUER"] = "1" if kernel == "halfpv" else "0"
+    if kernel not in ("half", "halfpv"):
         env["MLA_ATTN_KERNEL"] = kernel
     cases = CASES if cases is None else cases
     peaked = PEAKED if peaked is None else peaked
@@ -163,7 +169,10 @@ def oracle_case(d, mask):
 
 
 def test_kernels_against_oracle_and_each_other(cuda_device, tmp_path):
-    outs = {k: run_child(k, str(tmp_path / f"{k}.pt")) for k in ("half", "tile", "pair")}
+    outs = {k: run_child(k, str(tmp_path / f"{k}.pt"))
+            for k in ("half", "halfpv", "tile", "pair")}
+    for tag in outs["half"]:
+        assert torch.equal(outs["halfpv"][tag], outs["half"][tag]), (tag, "issue orders differ")
     report = {}
     err2 = {"half": 0.0, "tile": 0.0}
     for kind, cases in (("r", CASES), ("p", PEAKED)):
@@ -238,7 +247,7 @@ def test_every_kernel_masks_and_rotary_against_oracle(cuda_device, tmp_path):
             ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
                                        d["mask"], d["softmax_scale"])
         want[tag] = (ref, fm, B, T)
-    for kernel in ("half", "tile", "pair"):
+    for kernel in ("half", "halfpv", "tile", "pair"):
         outs = run_child(kernel, str(tmp_path / f"x_{kernel}.pt"), extra=True, cases=[],
                          peaked=[])
         for tag, (ref, fm, B, T) in want.items():

@@ -53,10 +53,14 @@ print(json.dumps({"launch": st_launch, "status": status, "word": word, "status2"
 """
 
 
-def test_bounded_wait_times_out_and_context_survives():
+@pytest.mark.parametrize("pv_issuer", ["0", "1"])
+def test_bounded_wait_times_out_and_context_survives(pv_issuer):
+    """With one issuer per query tile, and with the PV products issued by a
+    thread of their own (which must see the abort while it polls)."""
     env = dict(os.environ)
     env["MLA_TEST_STALL_WAIT"] = "1"
     env["MLA_WAIT_LIMIT_NS"] = "200000000"
+    env["MLA_ATTN_PV_ISSUER"] = pv_issuer
     code = "ROOT = %r\n" % ROOT + CHILD
     res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
                          timeout=600)
