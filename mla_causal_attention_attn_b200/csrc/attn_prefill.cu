@@ -448,7 +448,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const __grid_constant__ CUtensorMap tmKp,
                             const __grid_constant__ CUtensorMap tmV,
                             const __grid_constant__ CUtensorMap tmOut, const AttnArgs args) {
-  static_assert(!(kMasked && kHalf), "half-tile scores serve the causal kernel only");
   static_assert(kHalf || !kPvIssuer, "the PV issuer serves half-tile scores");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint64_t q_full[2];     // query tile i is in shared memory
@@ -467,6 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint64_t never_bar;    // no thread ever arrives (failure-detection test)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int mask_n_act[2];  // half tiles under a mask: each query tile's active prefix
+  __shared__ int mask_half;      // ... and whether both are prefixes (else 128-key tiles)
 
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -568,10 +569,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  if constexpr (kMasked && kHalf) {
+    // Half tiles take a query tile's active key tiles as a prefix [0, n_act).
+    // Under an explicit mask warp 3 reads the tile classes of both query
+    // tiles (32 per ballot): n_act is the index of the first skipped tile,
+    // and the CTA keeps 128-key tiles if an active tile follows a skipped one
+    // in either query tile.
+    if (warp == 3) {
+      bool prefix = true;
+#pragma unroll 1
+      for (int i = 0; i < 2; ++i) {
+        int f = 0;
+        if (tiles.exists[i]) {
+          f = args.n_kv;
+          const uint8_t* cls = tiles.cls[i];
+          for (int base = 0; base < args.n_kv; base += 32) {
+            const int kt = base + lane;
+            const bool in = kt < args.n_kv;
+            const bool act = in && (cls == nullptr || cls[kt] != kTileSkip);
+            const unsigned am = __ballot_sync(0xffffffffu, act);
+            const unsigned im = __ballot_sync(0xffffffffu, in && !act);
+            if (f == args.n_kv && im != 0u) f = base + __ffs(int(im)) - 1;
+            if (f < args.n_kv) {
+              const int sh = f - base;  // f lies in this chunk or an earlier one
+              const unsigned later = sh <= 0 ? am : (am & (0xffffffffu << sh));
+              if (later != 0u) prefix = false;
+            }
+          }
+        }
+        if (lane == 0) mask_n_act[i] = f;
+      }
+      if (lane == 0) mask_half = prefix ? 1 : 0;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
+  // Half-tile scores (kHalf): always for causal and valid-length calls; under
+  // an explicit mask when both query tiles' active key tiles are prefixes.
+  // n_act: active key tiles of each query tile, visited [0, vis_end).
+  const bool half = kHalf && (!kMasked || mask_half != 0);
+  auto n_act_of = [&](int i) -> int {
+    if constexpr (kMasked) return mask_n_act[i];
+    return tiles.exists[i] ? min(tiles.qt[i] + 1, tiles.end) : 0;
+  };
+  const int vis_end = kMasked ? max(n_act_of(0), n_act_of(1)) : tiles.end;
 
   if (warp < 4) {
   // Warpgroup 0 (TMA producer, MMA issuer, two idle warps) hands registers
@@ -679,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&ring_empty[seq % kRing]);
       };
-      if constexpr (kHalf) {
+      if (half) {
         // Half tiles: sub-tile u = 2 kt + hb is keys kt*128 + 64 hb .. +63 of
         // this query tile's active key tiles 0 .. n_act-1 (a prefix of the
         // visited ones); its scores go to buffer hb (64 TMEM columns, P over
@@ -688,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // works on this one. S(u+2) reuses the buffer PV(u) reads; the tensor
         // pipe runs one thread's MMAs in order.
         constexpr uint32_t idesc_sh = idesc_bf16_f32(kBQ, kBKV / 2, false, false);
-        const int n_act = min(tiles.qt[qi] + 1, tiles.end);
+        const int n_act = n_act_of(qi);
         const int n_sub = 2 * n_act;
         auto issue_s = [&](int u) -> bool {
           const int kt = u >> 1, hb = u & 1;
@@ -734,8 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           release(vseq, true);
           return true;
         };
-        if (ok) ok = issue_s(0);
-        if (ok) ok = issue_s(1);
+        if (ok && n_sub > 0) ok = issue_s(0);
+        if (ok && n_sub > 0) ok = issue_s(1);
         if constexpr (kPvIssuer) {
           // PV(u) comes from warp 3; S(u+2) follows it into the buffer.
           (void)issue_pv;
@@ -756,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The visited key tile past this query tile's last one (causal: the
         // other query tile's diagonal) is released unused, block by block
         // once it has landed, after every block this tile used.
-        for (int kt = n_act; ok && kt < tiles.end; ++kt)
+        for (int kt = n_act; ok && kt < vis_end; ++kt)
           for (uint32_t i = 0; ok && i < uint32_t(kBlocksPerTile); ++i) {
             const uint32_t seq = kBlocksPerTile * uint32_t(kt) + i;
             ok = wait_block(seq, 13);
@@ -778,13 +821,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 0..63 and 64..127 are two 8 KB halves (LBO), 8-key groups 1 KB
             // apart (SBO). 16 keys per MMA = 8 packed TMEM columns of P.
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const uint32_t vb = block_addr(prev_base + 3 + half);
+            for (int vh = 0; vh < 2; ++vh) {
+              const uint32_t vb = block_addr(prev_base + 3 + vh);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t acc = (n_pv > 0 || half > 0 || kk > 0) ? 1u : 0u;
+                const uint32_t acc = (n_pv > 0 || vh > 0 || kk > 0) ? 1u : 0u;
                 const uint64_t vd = sdesc_sw128(vb + kk * 16 * 128, kBlock / 2, 1024);
-                mma_ts(o_tmem, s_tmem + (half * 4 + kk) * 8, vd, idesc_o, acc);
+                mma_ts(o_tmem, s_tmem + (vh * 4 + kk) * 8, vd, idesc_o, acc);
               }
             }
             ++n_pv;
@@ -849,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if constexpr (kPvIssuer) {
-    if (warp == 3 && lane == 0 && has_work) {
+    if (warp == 3 && lane == 0 && has_work && half) {
       // ------------------------------------------------------------ PV issuer
       // For each query tile in turn: once P(u) is written and the V block of
       // half tile u has landed, O += P(u) V, release the V block, and tell
@@ -863,7 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n_sub[2], next[2] = {0, 0};
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        n_sub[t] = tiles.exists[t] ? 2 * min(tiles.qt[t] + 1, tiles.end) : 0;
+        n_sub[t] = 2 * n_act_of(t);
       bool ok = true, issued_any = false;
       unsigned long long last = globaltimer_ns();
       while (ok && (next[0] < n_sub[0] || next[1] < n_sub[1])) {
@@ -969,10 +1012,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY;  // running max, log2 units
     float l = 0.f;        // running sum of p (fp32, unrounded)
     uint32_t n = 0;
-    if constexpr (kHalf) {
-      // Half tiles (causal kernel): 64 keys per step, the two score buffers
-      // of this query tile in turn.
-      const int n_sub = (has_work && tiles.exists[wi]) ? 2 * min(qt + 1, tiles.end) : 0;
+    if (half) {
+      // Half tiles: 64 keys per step, the two score buffers of this query
+      // tile in turn.
+      const int n_sub = (has_work && tiles.exists[wi]) ? 2 * n_act_of(wi) : 0;
       for (int u = 0; u < n_sub; ++u) {
         const int kt = u >> 1, hb = u & 1;
         const int k0 = kt * kBKV + 64 * hb;
@@ -988,22 +1031,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // keys c <= lim of the half tile: c + 64 hb <= r on the diagonal tile
         // (none for rows r < 64 in its second half), and none at or past the
-        // sequence's key count
-        const bool causal_tile = kt == qt;
-        const bool diag = causal_tile || n_keys - k0 < kBKV / 2;
-        const int lim = min(causal_tile ? r - 64 * hb : kBKV / 2 - 1, n_keys - 1 - k0);
+        // sequence's key count. Under a mask the tile's class gives the
+        // limit: the causal pattern as above, a prefix class its last key
+        // minus 64 hb; mixed tiles add their 64 mask entries.
         ScoreChunk<kMasked> sc;
-        sc.cls = kTileZero;
-        sc.row_valid = row_valid;
-        sc.mrow = nullptr;
-        sc.kvalid = args.T - k0;
-        sc.mask_vec = 0;
-        sc.diag_row = diag ? lim : kBKV;
+        bool diag, fast_route;
+        int lim;
+        if constexpr (kMasked) {
+          // A second half that starts at or past T (the last key tile, T not a
+          // multiple of 128) holds no keys: class zero, so no mask entry is
+          // read for it and the limit below cuts every key.
+          const uint8_t tile_cls = args.T - k0 <= 0 ? uint8_t(kTileZero)
+                                   : tiles.cls[wi] ? tiles.cls[wi][kt] : uint8_t(kTileMixed);
+          const bool causal_tile = tile_cls == kTileCausal;
+          const bool prefix_tile = tile_cls >= kTilePrefix;
+          diag = causal_tile || prefix_tile || args.T - k0 < kBKV / 2;
+          lim = min(causal_tile ? r - 64 * hb
+                                : (prefix_tile ? int(tile_cls) - kTilePrefix - 64 * hb : kBKV / 2 - 1),
+                    args.T - 1 - k0);
+          fast_route = (tile_cls == kTileZero || causal_tile || prefix_tile) && args.scale_log2 > 0.f;
+          sc.cls = row_valid ? tile_cls : uint8_t(kTileZero);
+          sc.row_valid = row_valid;
+          sc.mrow = mrow + (row_valid ? k0 : 0);
+          sc.kvalid = args.T - k0;
+          sc.mask_vec = args.mask_vec;
+          sc.diag_row = (causal_tile || prefix_tile) ? lim : kBKV;
+        } else {
+          const bool causal_tile = kt == qt;
+          diag = causal_tile || n_keys - k0 < kBKV / 2;
+          lim = min(causal_tile ? r - 64 * hb : kBKV / 2 - 1, n_keys - 1 - k0);
+          fast_route = args.scale_log2 > 0.f;
+          sc.cls = kTileZero;
+          sc.row_valid = row_valid;
+          sc.mrow = nullptr;
+          sc.kvalid = args.T - k0;
+          sc.mask_vec = 0;
+          sc.diag_row = diag ? lim : kBKV;
+        }
         // Before rescaling O the step waits for PV(u-1): at most one PV of
         // this query tile is outstanding here (S(u), awaited above, was issued
         // after PV(u-2)), so the parity of pv_done is unambiguous.
         if (!softmax_step<kMasked, kBKV / 2>(args, lane_base, colS + 64 * hb, colO, sc,
-                                             args.scale_log2 > 0.f, diag, lim, r, n, m, l,
+                                             fast_route, diag, lim, r, n, m, l,
                                              &pv_done[wi], (n - 1) & 1u, ctl)) {
           ok = false;
           break;
@@ -2009,17 +2078,22 @@ cudaError_t launch_attn_prefill(const void* q_nope, const void* q_pe, const void
       !make_map_3d(&tmKn, k_nope, kDN, T, BH) || !make_map_3d(&tmKp, k_pe, kDR, T, B) ||
       !make_map_3d(&tmV, v, kDV, T, BH, 64) || !make_map_3d(&tmOut, out, kH * kDV, T, B))
     return cudaErrorInvalidValue;
-  // causal and valid-length calls: half-tile scores unless MLA_ATTN_KERNEL=tile
-  const bool half = !mask && !tile_kernel_selected();
+  // half-tile scores unless MLA_ATTN_KERNEL=tile (under an explicit mask the
+  // kernel falls back to 128-key tiles per CTA where needed)
+  const bool half = !tile_kernel_selected();
   const bool pv = half && pv_issuer_for(T);
-  auto kern = mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, false, false>
-                             : mla_attn_prefill_kernel<true, false, false, false>)
-              : pv ? (rope_cs ? mla_attn_prefill_kernel<false, true, true, true>
-                              : mla_attn_prefill_kernel<false, false, true, true>)
-              : half ? (rope_cs ? mla_attn_prefill_kernel<false, true, true, false>
-                                : mla_attn_prefill_kernel<false, false, true, false>)
-                     : (rope_cs ? mla_attn_prefill_kernel<false, true, false, false>
-                                : mla_attn_prefill_kernel<false, false, false, false>);
+  auto kern = pv ? (mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, true, true>
+                                    : mla_attn_prefill_kernel<true, false, true, true>)
+                         : (rope_cs ? mla_attn_prefill_kernel<false, true, true, true>
+                                    : mla_attn_prefill_kernel<false, false, true, true>))
+              : half ? (mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, true, false>
+                                        : mla_attn_prefill_kernel<true, false, true, false>)
+                             : (rope_cs ? mla_attn_prefill_kernel<false, true, true, false>
+                                        : mla_attn_prefill_kernel<false, false, true, false>))
+                     : (mask ? (rope_cs ? mla_attn_prefill_kernel<true, true, false, false>
+                                        : mla_attn_prefill_kernel<true, false, false, false>)
+                             : (rope_cs ? mla_attn_prefill_kernel<false, true, false, false>
+                                        : mla_attn_prefill_kernel<false, false, false, false>));
   static ContextCache attr_done[16];  // index: mask + 2 rope + 4 half + 8 PV issuer
   cudaError_t e = ensure_smem_attr(
       reinterpret_cast<const void*>(kern), int(kSmemBytes),

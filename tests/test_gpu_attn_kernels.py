@@ -128,6 +128,22 @@ def EXTRA_INPUTS():
     d["pos"] = inputs.make_positions(2, 300, "random", seed=906)
     d["mask"] = inputs.keypad_mask(torch.tensor([300, 111]), 300)
     out["ropem2x300"] = d
+    # a skipped key tile inside a query tile's range: batch 0's query tiles
+    # 2 and 3 see key tiles 0, 2, 3 but not 1, so their CTA runs 128-key
+    # tiles while the others take half tiles; batch 1 skips its last key
+    # tile. T = 400: the last key tile's second half lies past T.
+    gm = torch.Generator().manual_seed(907)
+    m = torch.randn(2, 1, 400, 400, generator=gm)
+    m[0, 0, 256:, 128:256] = float("-inf")
+    m[1, 0, :, 384:] = float("-inf")
+    m = m.to(torch.bfloat16)
+    d = inputs.make_inputs(2, 400, seed=908, with_weight=False)
+    d["mask"] = m
+    out["gap2x400"] = d
+    d = dict(inputs.make_inputs(2, 400, seed=909, with_weight=False))
+    d["pos"] = inputs.make_positions(2, 400, "offset")
+    d["mask"] = m
+    out["ropegap2x400"] = d
     return out
 """
 exec(EXTRA_SRC)
@@ -234,8 +250,10 @@ def test_tile_mode_mask_forms_are_bit_exact(cuda_device, tmp_path):
 def test_every_kernel_masks_and_rotary_against_oracle(cuda_device, tmp_path):
     """The explicit-mask and rotary instances of each kernel setting (the
     CTA-pair kernel runs them too when selected) against the fp64 oracle: a
-    general additive mask, a causal key-padding mask, and the rotary call
-    with offset positions, and with random positions under a mask."""
+    general additive mask, a causal key-padding mask, a mask that skips a
+    key tile inside a query tile's range (those CTAs keep 128-key tiles in
+    the half-tile settings), and the rotary call with offset positions, and
+    with random positions under a mask."""
     want = {}
     for tag, d in EXTRA_INPUTS().items():
         B, _, T, _ = d["q_nope"].shape
