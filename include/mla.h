@@ -47,8 +47,9 @@
  *    of the library's module variables, kernel attributes.
  *  - Environment (each read once per process): MLA_WAIT_LIMIT_NS sets the
  *    bounded waits' limit in nanoseconds; MLA_ATTN_KERNEL selects the
- *    attention kernel: unset, the one-SM kernel with 64-key score halves for
- *    causal and valid-length calls (128-key tiles for explicit masks);
+ *    attention kernel: unset, the one-SM kernel with 64-key score halves
+ *    (under an explicit mask, 128-key tiles for the CTAs whose query tiles
+ *    skip a key tile before a used one);
  *    "tile", 128-key tiles for every call; "pair", the CTA-pair kernel for
  *    every call. The choice changes rounding order only: every setting
  *    meets the same tolerance. MLA_ATTN_PV_ISSUER ("1" or "0") overrides

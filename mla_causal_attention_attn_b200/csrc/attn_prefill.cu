@@ -44,15 +44,21 @@
 //                against the running max; the others two passes.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
 //
-// Half-tile scores (causal and valid-length calls): with 128-key tiles a
+// Half-tile scores (the default): with 128-key tiles a
 // query tile's chain S_j -> softmax_j -> PV_j -> S_{j+1} is serial, and the
 // tensor pipe idles whenever both softmax warpgroups are busy. There each
 // 128-column S buffer is split into two 64-key buffers, and an issuer runs
 // S(0), S(1), then PV(u), S(u+2) for every 64-key half tile u, so the scores
 // of the next half tile are computed while the softmax works on this one;
 // the softmax waits for PV(u-1) only before it rescales O. The O accumulators
-// and the K/V ring are unchanged. Explicit masks keep 128-key tiles (a query
-// tile there may skip key tiles in the middle of the visited ones).
+// and the K/V ring are unchanged. The issue order needs each query tile's
+// active key tiles to be a prefix of the visited ones: always true for
+// causal and valid-length calls. Under an explicit mask the CTA checks its
+// tile classes and keeps 128-key tiles when a query tile skips a key tile
+// that a later one of its key tiles follows (the half-tile issuers would
+// have to release the skipped tile's ring blocks in between); a mask
+// tile's class maps onto its two halves (zero; causal, limit r - 64 half;
+// prefix L, limit L - 64 half; mixed, its 64 entries).
 //
 // Separate PV issuer (half tiles, T >= kPvIssuerMinT unless MLA_ATTN_PV_ISSUER
 // says otherwise): an issuer that waits for a K block of S(u+2) cannot issue
@@ -1967,8 +1973,8 @@ __global__ void __launch_bounds__(256)
 
 // Which attention kernel runs (MLA_ATTN_KERNEL, read once): "pair" selects
 // the CTA-pair kernel; "tile" the one-SM kernel with 128-key score tiles for
-// causal and valid-length calls too; anything else the one-SM kernel, with
-// half-tile scores for causal and valid-length calls.
+// every call; anything else the one-SM kernel with half-tile scores (under
+// an explicit mask where the CTA's active key tiles allow it).
 bool kernel_env_is(const char* name) {
   const char* s = std::getenv("MLA_ATTN_KERNEL");
   return s && std::strcmp(s, name) == 0;

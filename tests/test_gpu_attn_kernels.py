@@ -2,8 +2,9 @@
 
 Causal and valid-length calls run, by MLA_ATTN_KERNEL (read once per
 process), the one-SM kernel with 64-key (half-tile) score buffers (the
-default), the same kernel on 128-key tiles ("tile", the tiles explicit masks
-always use), or the CTA-pair kernel ("pair"). The half-tile kernel issues
+default; under an explicit mask a CTA whose query tiles skip a key tile
+before a used one keeps 128-key tiles), the same kernel on 128-key tiles
+("tile"), or the CTA-pair kernel ("pair"). The half-tile kernel issues
 its PV products either from each query tile's MMA issuer ("half") or from a
 thread of their own ("halfpv"; MLA_ATTN_PV_ISSUER=1, the default from
 T = 4096 on). Each runs here in a child process with the variables set.
