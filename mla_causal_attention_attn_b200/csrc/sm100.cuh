@@ -154,7 +154,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// Same as mbar_wait, for all 32 lanes of a warp; the verdict is warp-uniform.
+// Same as mbar_wait, for all 32 lanes of a warp; the result is warp-uniform.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& ctl,
                                                uint32_t site) {
   bool ok = mbar_wait(bar, parity, ctl, site);
