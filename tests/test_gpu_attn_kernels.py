@@ -132,11 +132,14 @@ def EXTRA_INPUTS():
     # a skipped key tile inside a query tile's range: batch 0's query tiles
     # 2 and 3 see key tiles 0, 2, 3 but not 1, so their CTA runs 128-key
     # tiles while the others take half tiles; batch 1 skips its last key
-    # tile. T = 400: the last key tile's second half lies past T.
+    # tile, and its query tile 1 has no allowed key at all (its rows are
+    # written as zeros while query tile 0 of the same CTA runs). T = 400: the
+    # last key tile's second half lies past T.
     gm = torch.Generator().manual_seed(907)
     m = torch.randn(2, 1, 400, 400, generator=gm)
     m[0, 0, 256:, 128:256] = float("-inf")
     m[1, 0, :, 384:] = float("-inf")
+    m[1, 0, 128:256, :] = float("-inf")
     m = m.to(torch.bfloat16)
     d = inputs.make_inputs(2, 400, seed=908, with_weight=False)
     d["mask"] = m
