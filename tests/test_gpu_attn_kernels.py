@@ -277,3 +277,24 @@ def test_every_kernel_masks_and_rotary_against_oracle(cuda_device, tmp_path):
             rows = ~fm.any(axis=1)
             assert np.all(got[~rows] == 0.0), (kernel, tag)
             assert_parity(got[rows], ref[rows], f"{kernel} {tag}")
+
+
+def test_pv_issuer_bit_identical_at_full_size(cuda_device, tmp_path):
+    """B=1, T=4096 (where the separate PV issuer is the default), random and
+    peaked inputs, causal and valid-length forms: the two issue orders give
+    the same bits, and on the peaked inputs every allowed row is v_t to half
+    a bf16 ulp."""
+    cases, peaked = [(1, 4096)], [(1, 4096)]
+    outs = {k: run_child(k, str(tmp_path / f"full_{k}.pt"), cases=cases, peaked=peaked)
+            for k in ("half", "halfpv")}
+    for tag in outs["half"]:
+        assert torch.equal(outs["halfpv"][tag], outs["half"][tag]), (tag, "issue orders differ")
+    B, T = peaked[0]
+    d = inputs.make_peaked_inputs(B, T, seed=1400 + T + B)
+    lens = lens_of(B, T)
+    for form, mask in (("", None), ("v", varlen_mask(B, T, lens))):
+        rows = np.array([t for t in range(T) if form == "" or t < lens[0]])
+        ref, fm = oracle.attn_rows(d["q_nope"], d["q_pe"], d["k_nope"], d["k_pe"], d["v"],
+                                   mask, d["softmax_scale"], rows=[(0, int(t)) for t in rows])
+        got = to_f64(outs["halfpv"][f"p{B}x{T}{form}"]).reshape(B * T, -1)[rows]
+        assert_peaked(got, ref, np.arange(len(rows)), f"halfpv p{B}x{T}{form}")
