@@ -194,13 +194,14 @@ def test_attn_prefix_mask_tiles_all_rows(cuda_device):
     assert_parity(to_f64(out).reshape(B * T, -1), ref, "attn prefix mask")
 
 
-def test_attn_keypad_dense_mask_matches_varlen(cuda_device):
+@pytest.mark.parametrize("B,T,lens", [(3, 700, [700, 333, 129]), (2, 4096, [4096, 1937])])
+def test_attn_keypad_dense_mask_matches_varlen(cuda_device, B, T, lens):
     """Causal attention with key padding, once as a dense mask and once as
     valid_len, on inputs whose row i points at keys i and i+1: rows t < len
     give v_t within half a bf16 ulp in both forms, and every row matches the
-    oracle in both. (On 128-key tiles the two forms agree bit for bit outside
+    oracle in both. At T = 4096 both forms run half tiles with the separate
+    PV issuer. (On 128-key tiles the two forms agree bit for bit outside
     the query tile holding the last valid key: test_gpu_attn_kernels.py.)"""
-    B, T, lens = 3, 700, [700, 333, 129]
     d = inputs.make_peaked_inputs(B, T, seed=5)
     d["mask"] = _prefix_mask(B, T, lens, causal=True)
     g = to_dev(d, cuda_device)
