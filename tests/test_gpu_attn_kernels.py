@@ -148,6 +148,13 @@ def EXTRA_INPUTS():
     d["pos"] = inputs.make_positions(2, 400, "offset")
     d["mask"] = m
     out["ropegap2x400"] = d
+    # the smallest explicit masks: T = 1 (the second 64-key half of the only
+    # key tile lies past T) and T = 65 (it holds one key)
+    for T, seed in ((1, 910), (65, 911)):
+        d = inputs.make_inputs(1, T, seed=seed, with_weight=False)
+        gm = torch.Generator().manual_seed(seed + 100)
+        d["mask"] = (torch.randn(1, 1, T, T, generator=gm) * 2.0).to(torch.bfloat16)
+        out[f"gen1x{T}"] = d
     return out
 """
 exec(EXTRA_SRC)
