@@ -802,9 +802,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) mma_commit(&o_final[qi]);
         }
-        // The visited key tile past this query tile's last one (causal: the
-        // other query tile's diagonal) is released unused, block by block
-        // once it has landed, after every block this tile used.
+        // The visited key tiles past this query tile's last one (causal: the
+        // other query tile's diagonal; under a mask, up to the other query
+        // tile's prefix) are released unused, block by block once landed,
+        // after every block this tile used.
         for (int kt = n_act; ok && kt < vis_end; ++kt)
           for (uint32_t i = 0; ok && i < uint32_t(kBlocksPerTile); ++i) {
             const uint32_t seq = kBlocksPerTile * uint32_t(kt) + i;
